@@ -1,0 +1,190 @@
+/*
+ * attn.h -- C ABI of the B200 (sm_100a) exact-attention library with a KV cache.
+ *
+ * The library computes softmax(scale * Q K^T) V tile by tile with an online
+ * softmax (running maximum m, running denominator l, rescale when m grows), so
+ * the score matrix never reaches HBM; decode splits the keys into chunks that
+ * are processed in parallel and merged by a log-sum-exp combine.
+ *
+ * Source pages (cited by title and section):
+ *   [P1] "KV cache, flash attention and inference optimisation" lesson
+ *        (AI Engineering from Scratch, Phase 07 · 12)
+ *   [P2] "大模型面试笔记——Attention篇" (juejin)
+ *   [P3] "[BEE-30062] FlashAttention 與高效注意力核心"
+ *   [P5] "Effizienz" chapter (tokenwerk)
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are dense, row-major and token-major ("BSHD"), the layout of the
+ *     [P3] "為長上下文推論啟用 FlashDecoding" section: q (batch, tokens, q_heads,
+ *     head_dim), caches (batch, seqlen_cache, kv_heads, head_dim).
+ *   - bf16 is IEEE bfloat16 stored as 2-byte little-endian words.
+ *   - GQA/MQA: query head h reads K/V head h / (Hq / Hkv) ([P5] "GQA im leicht
+ *     lesbaren Code": repeat_interleave along the head axis).  Hq % Hkv == 0.
+ *   - Head dimension d is 64 or 128.
+ *   - LSE outputs are natural-log log-sum-exp of the SCALED scores, fp32.
+ *   - Paged caches ([P1] "页面注意 KV缓存作为虚拟内存"): pools of 16-token physical
+ *     blocks laid out [num_blocks, 16, Hkv, d]; a page table int32
+ *     [B, max_blocks_per_seq] maps logical block j/16 of sequence b to a
+ *     physical block; token j sits in slot j % 16.
+ *   - Pointers named "device" must be device (or managed) memory of the current
+ *     device; the caller owns every buffer, including the decode workspace.  The
+ *     library allocates nothing per call.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and returns a status.  Host-side argument checks run
+ *     before anything is launched and return a negative status.  Checks that
+ *     need device data (lengths, page ids) set bits of a sticky device status
+ *     word instead of faulting; read it with attn_get_device_status().
+ */
+#ifndef KVATTN_ATTN_H
+#define KVATTN_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- return codes -------------------------------------------------------- */
+enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = -1, /* null pointer, inconsistent or non-positive sizes, bad dtype */
+  ATTN_ERR_UNSUPPORTED = -2, /* valid request outside what is built (d, rows per KV head) */
+  ATTN_ERR_WORKSPACE = -3,   /* decode workspace missing or smaller than required */
+  ATTN_ERR_CUDA = -4,        /* a CUDA runtime/driver call failed (launch, tensor map, ...) */
+  ATTN_ERR_DEVICE = -5       /* the device status word is non-zero (attn_get_device_status) */
+};
+
+/* ---- output element types ------------------------------------------------ */
+enum { ATTN_F32 = 0, ATTN_BF16 = 1 };
+
+/* ---- device status bits (sticky until cleared) --------------------------- */
+enum {
+  ATTN_DEV_PAGE_ID = 1,      /* a page-table entry read was outside [0, num_blocks) */
+  ATTN_DEV_SEQLEN = 2,       /* seqlens_k[b] < T, > max_seqlen_k or beyond the cache capacity */
+  ATTN_DEV_APPEND_RANGE = 4, /* kv_append position beyond the cache capacity / page table */
+  ATTN_DEV_TIMEOUT = 8       /* a bounded wait inside a kernel gave up (no fault, results invalid) */
+};
+
+/*
+ * attn_prefill -- exact attention over a whole prompt, Nq == Nk == N.
+ *
+ * Defines: [P1] "片技巧" (standard attention S = Q K^T, P = softmax(S), O = P V,
+ * computed per Q tile against K/V tiles with a running softmax so the N x N
+ * matrix never reaches HBM) and [P2] section 2 (online safe softmax: keep the
+ * running maximum m and denominator l, multiply l by a compensation factor when
+ * m changes).  causal = 1 is [P3]'s SDPA is_causal: query i sees keys j <= i.
+ *
+ *   q    device bf16 [B, N, Hq, d]
+ *   k, v device bf16 [B, N, Hkv, d]
+ *   o    device [B, N, Hq, d], element type o_dtype (ATTN_F32 or ATTN_BF16)
+ *   lse  device fp32 [B, Hq, N], or NULL to skip
+ *   scale  multiplies q.k (e.g. 1/sqrt(d)); must be finite and > 0
+ *   causal 0 or 1
+ * Errors: ATTN_ERR_INVALID_ARG for null pointers / sizes < 1 / Hq % Hkv;
+ * ATTN_ERR_UNSUPPORTED for d not in {64, 128}; ATTN_ERR_CUDA on launch failure.
+ * Runs on tcgen05 tensor cores with TMEM accumulators and TMA-staged tiles.
+ */
+ATTN_API int attn_prefill(const void* q, const void* k, const void* v, void* o, int o_dtype, float* lse, int B, int Hq,
+                 int Hkv, int N, int d, float scale, int causal, void* stream);
+
+/*
+ * attn_decode_workspace_bytes -- bytes of device workspace attn_decode needs
+ * for these sizes (the per-chunk partial outputs and log-sum-exps of the split
+ * along the keys).  num_splits as for attn_decode.  Returns 0 for invalid sizes.
+ */
+ATTN_API size_t attn_decode_workspace_bytes(int B, int T, int Hq, int Hkv, int d, int max_seqlen_k, int num_splits);
+
+/*
+ * attn_decode -- T new query tokens per sequence against a KV cache.
+ *
+ * Defines: [P2] section 4 (next-token output softmax(t_Q x_K^T / sqrt(h)) x_V
+ * over every cached key: no Q cache, O(N) per step), [P3] "背景" and
+ * "為長上下文推論啟用 FlashDecoding" (Flash-Decoding: the keys are split into
+ * chunks processed in parallel and the partial softmax results are reduced in a
+ * numerically stable way; arguments q, k_cache, v_cache, cache_seqlens,
+ * causal), and [P5] "Der wichtige Maskenfehler beim Cache" (the new queries are
+ * the LAST T positions: with causal = 1, token t of T sees keys
+ * j <= seqlens_k[b] - T + t; a single new token sees the whole cache).
+ *
+ *   q           device bf16 [B, T, Hq, d]
+ *   k_cache,    contiguous (page_table == NULL): device bf16 [B, cache_capacity, Hkv, d]
+ *   v_cache     paged: device bf16 pools [num_blocks, 16, Hkv, d]
+ *   seqlens_k   device int32 [B]: valid keys of sequence b, INCLUDING the T new
+ *               tokens (append them with kv_append first, on the same stream)
+ *   page_table  device int32 [B, max_blocks_per_seq], or NULL for a contiguous cache
+ *   max_blocks_per_seq, num_blocks   paged sizes (ignored when contiguous)
+ *   cache_capacity  contiguous token capacity per sequence (ignored when paged)
+ *   max_seqlen_k    host-side upper bound on every seqlens_k[b] (sizes the split
+ *                   grid and the workspace); 0 = the cache capacity
+ *   o           device [B, T, Hq, d] of o_dtype;  lse  device fp32 [B, Hq, T] or NULL
+ *   scale, causal   as for attn_prefill; causal with T == 1 equals non-causal
+ *   num_splits  0 = automatic chunking; n > 0 = split every sequence's keys
+ *               into at most n chunks
+ *   workspace   device memory of at least attn_decode_workspace_bytes(...) bytes,
+ *               16-byte aligned; contents on entry do not matter
+ * Rows per KV head (Hq / Hkv) * T must be <= 32.
+ * Errors: ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED (d, rows per KV head),
+ * ATTN_ERR_WORKSPACE, ATTN_ERR_CUDA.  Bad lengths or page ids found on the
+ * device set ATTN_DEV_SEQLEN / ATTN_DEV_PAGE_ID and make the affected rows NaN.
+ */
+ATTN_API int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens_k,
+                const int32_t* page_table, int max_blocks_per_seq, int num_blocks, int cache_capacity,
+                int max_seqlen_k, void* o, int o_dtype, float* lse, int B, int T, int Hq, int Hkv, int d,
+                float scale, int causal, int num_splits, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * kv_append -- write the K and V rows of T new tokens into the cache.
+ *
+ * Defines: [P2] section 4, x_K <- Concat(x_K, t W_K) and x_V <- Concat(x_V, t W_V)
+ * (the projections t W are the caller's), and [P1] "步骤1" (the cache grows by
+ * one K,V vector per token per layer per head).  Token t of sequence b goes to
+ * position p = cache_lens[b] + t: contiguous row p, or paged block
+ * page_table[b][p / 16], slot p % 16.
+ *
+ *   k_cache, v_cache  as for attn_decode (written)
+ *   k_new, v_new      device bf16 [B, T, Hkv, d]
+ *   cache_lens        device int32 [B]: lengths BEFORE the append (not modified;
+ *                     the caller advances them)
+ *   page_table, max_blocks_per_seq, num_blocks, cache_capacity  as for attn_decode
+ * Errors: ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED (d), ATTN_ERR_CUDA.  A
+ * position beyond the capacity / page table, or a bad page id, is skipped and
+ * sets ATTN_DEV_APPEND_RANGE / ATTN_DEV_PAGE_ID.
+ */
+ATTN_API int kv_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new, const int32_t* cache_lens,
+              const int32_t* page_table, int max_blocks_per_seq, int num_blocks, int cache_capacity, int B, int T,
+              int Hkv, int d, void* stream);
+
+/*
+ * kv_cache_bytes -- bytes held by a KV cache: 2 * n_layers * batch * tokens *
+ * n_kv_heads * head_dim * elem_bytes, the K and V factor times every dimension.
+ *
+ * Defines: [P5] "Cachebedarf berechnen" (worked example L=6, B=1, T=1024,
+ * Hkv=2, d=64, e=2 gives 3,145,728 bytes) and [P1] "预存计算" (bytes per token
+ * per layer = 2 * n_kv_heads * d_head * dtype_size).  Host only, exact integer
+ * arithmetic.  Returns -1 if any argument is <= 0 or the product overflows int64.
+ */
+ATTN_API int64_t kv_cache_bytes(int n_layers, int batch, int64_t tokens, int n_kv_heads, int head_dim, int elem_bytes);
+
+/*
+ * attn_get_device_status -- OR of the ATTN_DEV_* bits set by kernels on the
+ * current device since the last clear.  Synchronises the device.  clear != 0
+ * resets the word to 0 after reading.  Returns ATTN_ERR_CUDA (negative) if the
+ * word cannot be read.  Not part of the pages' method: error reporting only.
+ */
+ATTN_API int attn_get_device_status(int clear);
+
+/* attn_status_string -- static text for a return code (never NULL). */
+ATTN_API const char* attn_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVATTN_ATTN_H */

@@ -1,0 +1,180 @@
+"""Exact attention with a KV cache on NVIDIA B200 (sm_100a).
+
+Python binding of ``libkvattn.so``: the functions below carry the C-ABI names of
+``include/attn.h`` and only marshal arguments (device pointers, sizes, the
+current CUDA stream) from torch tensors.  Every step of the computation runs in
+the library's CUDA kernels; there is no CPU or library fallback, and importing
+this package fails if the library has not been built
+(``python -m kv_cache_decode_attn_b200.build``).
+
+The raw ctypes handle is ``lib``; tests call through it or through these wrappers.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+__all__ = [
+    "lib", "LIB_PATH", "AttnError",
+    "attn_prefill", "attn_decode", "attn_decode_workspace_bytes", "kv_append", "kv_cache_bytes",
+    "attn_get_device_status", "attn_status_string", "decode_workspace",
+    "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_WORKSPACE", "ATTN_ERR_CUDA",
+    "ATTN_ERR_DEVICE", "ATTN_F32", "ATTN_BF16", "ATTN_DEV_PAGE_ID", "ATTN_DEV_SEQLEN",
+    "ATTN_DEV_APPEND_RANGE", "ATTN_DEV_TIMEOUT",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvattn.so")
+
+ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_WORKSPACE, ATTN_ERR_CUDA, ATTN_ERR_DEVICE = 0, -1, -2, -3, -4, -5
+ATTN_F32, ATTN_BF16 = 0, 1
+ATTN_DEV_PAGE_ID, ATTN_DEV_SEQLEN, ATTN_DEV_APPEND_RANGE, ATTN_DEV_TIMEOUT = 1, 2, 4, 8
+
+_p, _i, _i64, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+
+_SIGNATURES = {
+    "attn_prefill": (_i, [_p, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _f, _i, _p]),
+    "attn_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "attn_decode": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _p, _i, _p, _i, _i, _i, _i, _i, _f, _i, _i, _p, _sz,
+                         _p]),
+    "kv_append": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p]),
+    "kv_cache_bytes": (_i64, [_i, _i, _i64, _i, _i, _i]),
+    "attn_get_device_status": (_i, [_i]),
+    "attn_status_string": (ctypes.c_char_p, [_i]),
+}
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m kv_cache_decode_attn_b200.build`")
+    handle = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(handle, name)
+        fn.restype = res
+        fn.argtypes = args
+    return handle
+
+
+lib = _load()
+
+
+class AttnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: {attn_status_string(status)} ({status})")
+        self.status = status
+
+
+def attn_status_string(status: int) -> str:
+    return lib.attn_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != ATTN_OK:
+        raise AttnError(fn, status)
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}")
+    return t.data_ptr()
+
+
+def _out_dtype(o: torch.Tensor) -> int:
+    if o.dtype == torch.float32:
+        return ATTN_F32
+    if o.dtype == torch.bfloat16:
+        return ATTN_BF16
+    raise ValueError("output must be float32 or bfloat16")
+
+
+def attn_prefill(q, k, v, o, lse=None, scale=None, causal=True, stream=None) -> None:
+    """q ``[B, N, Hq, d]``, k/v ``[B, N, Hkv, d]`` bf16 -> o ``[B, N, Hq, d]`` (f32 or bf16),
+    lse ``[B, Hq, N]`` f32 (optional)."""
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if tuple(k.shape) != (B, N, Hkv, d) or tuple(v.shape) != tuple(k.shape) or tuple(o.shape) != (B, N, Hq, d):
+        raise ValueError("shape mismatch")
+    if lse is not None and tuple(lse.shape) != (B, Hq, N):
+        raise ValueError("lse must be [B, Hq, N]")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    st = lib.attn_prefill(_dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16), _dev(v, "v", torch.bfloat16),
+                          _dev(o, "o"), _out_dtype(o), None if lse is None else _dev(lse, "lse", torch.float32),
+                          B, Hq, Hkv, N, d, scale, int(bool(causal)), _stream(stream))
+    _check("attn_prefill", st)
+
+
+def attn_decode_workspace_bytes(B, T, Hq, Hkv, d, max_seqlen_k, num_splits=0) -> int:
+    return int(lib.attn_decode_workspace_bytes(B, T, Hq, Hkv, d, max_seqlen_k, num_splits))
+
+
+def decode_workspace(B, T, Hq, Hkv, d, max_seqlen_k, num_splits=0, device="cuda") -> torch.Tensor:
+    """Caller-owned workspace for ``attn_decode`` (allocated by torch)."""
+    n = attn_decode_workspace_bytes(B, T, Hq, Hkv, d, max_seqlen_k, num_splits)
+    if n == 0:
+        raise ValueError("invalid decode sizes")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def _cache_geometry(k_cache, page_table):
+    if page_table is None:
+        return 0, 0, int(k_cache.shape[1]), int(k_cache.shape[2])
+    return int(page_table.shape[1]), int(k_cache.shape[0]), 0, int(k_cache.shape[2])
+
+
+def attn_decode(q, k_cache, v_cache, seqlens_k, o, lse=None, page_table=None, max_seqlen_k=0, scale=None,
+                causal=True, num_splits=0, workspace=None, stream=None) -> None:
+    """q ``[B, T, Hq, d]``; k/v cache ``[B, cap, Hkv, d]`` or pools ``[nblk, 16, Hkv, d]``;
+    seqlens_k int32 ``[B]`` (including the T new tokens); page_table int32 ``[B, max_blocks]``."""
+    B, T, Hq, d = q.shape
+    max_blocks, num_blocks, cap, Hkv = _cache_geometry(k_cache, page_table)
+    if tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(o.shape) != (B, T, Hq, d):
+        raise ValueError("shape mismatch")
+    if lse is not None and tuple(lse.shape) != (B, Hq, T):
+        raise ValueError("lse must be [B, Hq, T]")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if workspace is None:
+        msk = max_seqlen_k if max_seqlen_k else (cap if page_table is None else max_blocks * 16)
+        workspace = decode_workspace(B, T, Hq, Hkv, d, msk, num_splits, q.device)
+    st = lib.attn_decode(_dev(q, "q", torch.bfloat16), _dev(k_cache, "k_cache", torch.bfloat16),
+                         _dev(v_cache, "v_cache", torch.bfloat16), _dev(seqlens_k, "seqlens_k", torch.int32),
+                         None if page_table is None else _dev(page_table, "page_table", torch.int32),
+                         max_blocks, num_blocks, cap, int(max_seqlen_k), _dev(o, "o"), _out_dtype(o),
+                         None if lse is None else _dev(lse, "lse", torch.float32), B, T, Hq, Hkv, d, scale,
+                         int(bool(causal)), int(num_splits), _dev(workspace, "workspace"),
+                         workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("attn_decode", st)
+
+
+def kv_append(k_cache, v_cache, k_new, v_new, cache_lens, page_table=None, stream=None) -> None:
+    """Write k_new/v_new ``[B, T, Hkv, d]`` at positions cache_lens[b] + t (cache_lens int32, before the append)."""
+    B, T, Hkv, d = k_new.shape
+    max_blocks, num_blocks, cap, Hkv_c = _cache_geometry(k_cache, page_table)
+    if Hkv_c != Hkv or tuple(v_new.shape) != tuple(k_new.shape) or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("shape mismatch")
+    st = lib.kv_append(_dev(k_cache, "k_cache", torch.bfloat16), _dev(v_cache, "v_cache", torch.bfloat16),
+                       _dev(k_new, "k_new", torch.bfloat16), _dev(v_new, "v_new", torch.bfloat16),
+                       _dev(cache_lens, "cache_lens", torch.int32),
+                       None if page_table is None else _dev(page_table, "page_table", torch.int32),
+                       max_blocks, num_blocks, cap, B, T, Hkv, d, _stream(stream))
+    _check("kv_append", st)
+
+
+def kv_cache_bytes(n_layers, batch, tokens, n_kv_heads, head_dim, elem_bytes) -> int:
+    return int(lib.kv_cache_bytes(n_layers, batch, tokens, n_kv_heads, head_dim, elem_bytes))
+
+
+def attn_get_device_status(clear: bool = False) -> int:
+    return int(lib.attn_get_device_status(int(bool(clear))))

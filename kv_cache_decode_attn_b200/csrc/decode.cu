@@ -1,0 +1,520 @@
+// Split-KV decode attention for sm_100a (memory-bound path).
+//
+// One CTA owns one work item (sequence b, KV head g, key chunk c).  All
+// R = (Hq/Hkv) * T query rows that read KV head g are handled together, so each
+// K/V byte is streamed from HBM once per step.  A producer warp moves 64-token
+// K/V tiles into a shared-memory ring with TMA (128-byte swizzle, evict-first
+// L2 policy); consumer warps compute S = Q K^T and O += P V with warp-level bf16
+// tensor-core MMAs (fp32 accumulation), keeping a running maximum and running
+// denominator per row and rescaling O when the maximum grows.  Each consumer
+// warp owns 16 tokens of every tile, so the four warps of a row group are four
+// independent online softmaxes that are merged at the end of the chunk.  The
+// chunk's normalised output and log-sum-exp go to the workspace; a second
+// kernel merges the chunks of each row with the log-sum-exp combine.
+//
+// Method: "[BEE-30062] FlashAttention 與高效注意力核心", sections "背景" and
+// "為長上下文推論啟用 FlashDecoding" (split along the KV length, numerically
+// stable reduction of partial softmax results); "大模型面試笔记——Attention篇"
+// section 2 (online safe softmax); "Effizienz", "Der wichtige Maskenfehler beim
+// Cache" (bottom-right aligned mask for several new tokens).
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace kvattn {
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+template <int D, int MT>
+struct DecodeCfg {
+  static constexpr int kConsumerWarps = 4 * MT;
+  static constexpr int kThreads = 32 * (kConsumerWarps + 1);
+  static constexpr int kHalves = D / 64;              // 128-byte swizzle spans 64 bf16
+  static constexpr int kHalfBytes = kDecodeTile * 128;
+  static constexpr int kTensorBytes = kHalves * kHalfBytes;   // one of K or V per stage
+  static constexpr int kStageBytes = 2 * kTensorBytes;
+  static constexpr int kStages = (MT == 1) ? (D == 128 ? 3 : 6) : (D == 128 ? 4 : 8);
+  static constexpr int kRedStride = D + 8;            // floats per row of the merge buffer
+  static constexpr int kRedBytes = MT * 4 * 16 * kRedStride * 4;
+  static_assert(kRedBytes <= kStages * kStageBytes, "merge buffer must fit in the ring");
+  static constexpr int kBarOffset = kStages * kStageBytes;
+  static constexpr int kStatsOffset = kBarOffset + 2 * kStages * 8;
+  static constexpr int kSmemBytes = kStatsOffset + MT * 4 * 16 * 2 * 4 + 16 + 1024;  // + alignment slack
+  static constexpr int kMinBlocks = (kSmemBytes * 2 <= 227 * 1024) ? 2 : 1;
+};
+
+struct SplitParams {
+  const __nv_bfloat16* q;
+  const int32_t* seqlens;
+  const int32_t* page_table;
+  float* part_o;
+  float* part_lse;
+  unsigned* status;
+  int T, Hq, Hkv, G, R;
+  int chunk, max_chunks, capacity, max_blocks, num_blocks, max_seqlen;
+  float scale_log2;
+  int causal;
+};
+
+__device__ __forceinline__ bool seqlen_bad(int L, int T, int max_seqlen, bool paged, int capacity, int max_blocks) {
+  if (L < T || L > max_seqlen) return true;
+  if (!paged && L > capacity) return true;
+  if (paged && (L + kPageTokens - 1) / kPageTokens > max_blocks) return true;
+  return false;
+}
+
+template <int D, int MT, bool PAGED>
+__global__ void __launch_bounds__(DecodeCfg<D, MT>::kThreads, DecodeCfg<D, MT>::kMinBlocks)
+    decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                        const SplitParams p) {
+  using C = DecodeCfg<D, MT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
+  uint64_t* empty = full + C::kStages;
+  float* stats = reinterpret_cast<float*>(smem + C::kStatsOffset);   // [MT][4][16][2]: m, l
+  int* abort_flag = reinterpret_cast<int*>(stats + MT * 4 * 16 * 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+
+  const int L = p.seqlens[b];
+  if (seqlen_bad(L, p.T, p.max_seqlen, PAGED, p.capacity, p.max_blocks)) {
+    if (threadIdx.x == 0 && c == 0 && g == 0) atomicOr(p.status, DEV_SEQLEN);
+    return;   // the combine kernel writes NaN rows for this sequence
+  }
+  const int tok_begin = c * p.chunk;
+  if (tok_begin >= L) return;
+  const int tok_end = min(tok_begin + p.chunk, L);
+  const int n_tiles = (tok_end - tok_begin + kDecodeTile - 1) / kDecodeTile;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], C::kConsumerWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == C::kConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      const uint64_t pol = policy_evict_first();
+      for (int i = 0; i < n_tiles; ++i) {
+        const int s = i % C::kStages;
+        if (i >= C::kStages && !mbar_wait(&empty[s], ((i / C::kStages) - 1) & 1)) {
+          atomicOr(p.status, DEV_TIMEOUT);
+          *reinterpret_cast<volatile int*>(abort_flag) = 1;
+          break;
+        }
+        uint8_t* kst = smem + s * C::kStageBytes;
+        uint8_t* vst = kst + C::kTensorBytes;
+        const int t0 = tok_begin + i * kDecodeTile;
+        if (!PAGED) {
+          mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+          const int row = b * p.capacity + t0;
+#pragma unroll
+          for (int h = 0; h < C::kHalves; ++h) {
+            tma_load_3d(kst + h * C::kHalfBytes, &tmK, &full[s], h * 64, g, row, pol);
+            tma_load_3d(vst + h * C::kHalfBytes, &tmV, &full[s], h * 64, g, row, pol);
+          }
+        } else {
+          const int nb = min(kDecodeTile / kPageTokens, (tok_end - t0 + kPageTokens - 1) / kPageTokens);
+          mbar_arrive_expect_tx(&full[s], nb * 2 * C::kHalves * kPageTokens * 128);
+          const int32_t* row_tab = p.page_table + (size_t)b * p.max_blocks + t0 / kPageTokens;
+          for (int j = 0; j < nb; ++j) {
+            int blk = row_tab[j];
+            if (blk < 0 || blk >= p.num_blocks) {
+              atomicOr(p.status, DEV_PAGE_ID);
+              blk = 0;   // keep the byte count; the result is flagged invalid
+            }
+#pragma unroll
+            for (int h = 0; h < C::kHalves; ++h) {
+              tma_load_3d(kst + h * C::kHalfBytes + j * kPageTokens * 128, &tmK, &full[s], h * 64, g,
+                          blk * kPageTokens, pol);
+              tma_load_3d(vst + h * C::kHalfBytes + j * kPageTokens * 128, &tmV, &full[s], h * 64, g,
+                          blk * kPageTokens, pol);
+            }
+          }
+        }
+      }
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int wsub = warp & 3;          // which 16 tokens of each tile
+  const int mt = warp >> 2;           // which 16 query rows
+  const int gid = lane >> 2, tig = lane & 3;
+
+  // Query rows r0 = mt*16 + gid and r1 = r0 + 8; row r is (token t = r / G, head g*G + r % G).
+  const int r0 = mt * 16 + gid, r1 = r0 + 8;
+  int end0 = L, end1 = L;   // first invisible key of each row
+  if (p.causal) {
+    if (r0 < p.R) end0 = L - p.T + r0 / p.G + 1;
+    if (r1 < p.R) end1 = L - p.T + r1 / p.G + 1;
+  }
+
+  // Q fragments (A operand, 16 x D, row-major) straight from global memory.
+  uint32_t qa[D / 16][4];
+  {
+    auto qrow = [&](int r) -> const __nv_bfloat16* {
+      const int t = r / p.G, hh = r - t * p.G;
+      return p.q + (((size_t)b * p.T + t) * p.Hq + (size_t)g * p.G + hh) * D;
+    };
+    const __nv_bfloat16* qr0 = r0 < p.R ? qrow(r0) : nullptr;
+    const __nv_bfloat16* qr1 = r1 < p.R ? qrow(r1) : nullptr;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int c0 = kk * 16 + tig * 2;
+      qa[kk][0] = qr0 ? *reinterpret_cast<const uint32_t*>(qr0 + c0) : 0u;
+      qa[kk][1] = qr1 ? *reinterpret_cast<const uint32_t*>(qr1 + c0) : 0u;
+      qa[kk][2] = qr0 ? *reinterpret_cast<const uint32_t*>(qr0 + c0 + 8) : 0u;
+      qa[kk][3] = qr1 ? *reinterpret_cast<const uint32_t*>(qr1 + c0 + 8) : 0u;
+    }
+  }
+
+  float o_acc[D / 8][4];
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) o_acc[n][0] = o_acc[n][1] = o_acc[n][2] = o_acc[n][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+  // ldmatrix lane roles
+  const int lm = lane >> 3, lr = lane & 7;
+  bool aborted = false;
+
+  for (int i = 0; i < n_tiles; ++i) {
+    const int s = i % C::kStages;
+    if (!mbar_wait(&full[s], (i / C::kStages) & 1)) {
+      atomicOr(p.status, DEV_TIMEOUT);
+      aborted = true;
+      break;
+    }
+    if (*reinterpret_cast<volatile int*>(abort_flag)) { aborted = true; break; }
+    const uint32_t kbase = smem_u32(smem + s * C::kStageBytes);
+    const uint32_t vbase = kbase + C::kTensorBytes;
+    const int tok_base = tok_begin + i * kDecodeTile + wsub * 16;
+
+    // ---- S = Q K^T for this warp's 16 tokens (two n8 tiles)
+    float sacc[2][4];
+#pragma unroll
+    for (int n = 0; n < 2; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
+    {
+      const int trow = wsub * 16 + (lm >> 1) * 8 + lr;   // token row inside the tile
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const int chunk16 = kk * 2 + (lm & 1);             // 16-byte chunk along d
+        const int h = chunk16 >> 3, cw = chunk16 & 7;
+        const uint32_t addr = kbase + h * C::kHalfBytes + trow * 128 + ((cw ^ (trow & 7)) << 4);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(addr, b0, b1, b2, b3);
+        mma_bf16_16816(sacc[0], qa[kk], b0, b1);
+        mma_bf16_16816(sacc[1], qa[kk], b2, b3);
+      }
+    }
+
+    // ---- online softmax (base-2 exponent, scale folded in)
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int n = 0; n < 2; ++n) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int tok = tok_base + n * 8 + tig * 2 + (e & 1);
+        const int end = (e < 2) ? end0 : end1;
+        const float v = (tok < end) ? sacc[n][e] * p.scale_log2 : -INFINITY;
+        sacc[n][e] = v;
+        if (e < 2) mx0 = fmaxf(mx0, v); else mx1 = fmaxf(mx1, v);
+      }
+    }
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+    const float mu0 = (mn0 == -INFINITY) ? 0.f : mn0;
+    const float mu1 = (mn1 == -INFINITY) ? 0.f : mn1;
+    const float al0 = ex2(m0 - mu0), al1 = ex2(m1 - mu1);
+    m0 = mn0;
+    m1 = mn1;
+    float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+    for (int n = 0; n < 2; ++n) {
+      sacc[n][0] = ex2(sacc[n][0] - mu0);
+      sacc[n][1] = ex2(sacc[n][1] - mu0);
+      sacc[n][2] = ex2(sacc[n][2] - mu1);
+      sacc[n][3] = ex2(sacc[n][3] - mu1);
+      ps0 += sacc[n][0] + sacc[n][1];
+      ps1 += sacc[n][2] + sacc[n][3];
+    }
+    l0 = l0 * al0 + ps0;
+    l1 = l1 * al1 + ps1;
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      o_acc[n][0] *= al0;
+      o_acc[n][1] *= al0;
+      o_acc[n][2] *= al1;
+      o_acc[n][3] *= al1;
+    }
+    uint32_t pa[4];
+    pa[0] = pack_bf16x2(sacc[0][0], sacc[0][1]);
+    pa[1] = pack_bf16x2(sacc[0][2], sacc[0][3]);
+    pa[2] = pack_bf16x2(sacc[1][0], sacc[1][1]);
+    pa[3] = pack_bf16x2(sacc[1][2], sacc[1][3]);
+
+    // ---- O += P V ; keys at or past L may hold anything (even NaN): zero them
+    const bool tail = tok_base + 16 > L;
+    const int vrow = wsub * 16 + (lm & 1) * 8 + lr;
+#pragma unroll
+    for (int nn = 0; nn < D / 16; ++nn) {
+      const int chunk16 = nn * 2 + (lm >> 1);
+      const int h = chunk16 >> 3, cw = chunk16 & 7;
+      const uint32_t addr = vbase + h * C::kHalfBytes + vrow * 128 + ((cw ^ (vrow & 7)) << 4);
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(addr, b0, b1, b2, b3);
+      if (tail) {
+        const int ta = tok_base + tig * 2, tb = ta + 8;
+        const uint32_t mlo_a = (ta < L) ? 0x0000ffffu : 0u, mhi_a = (ta + 1 < L) ? 0xffff0000u : 0u;
+        const uint32_t mlo_b = (tb < L) ? 0x0000ffffu : 0u, mhi_b = (tb + 1 < L) ? 0xffff0000u : 0u;
+        b0 &= (mlo_a | mhi_a);
+        b2 &= (mlo_a | mhi_a);
+        b1 &= (mlo_b | mhi_b);
+        b3 &= (mlo_b | mhi_b);
+      }
+      mma_bf16_16816(o_acc[2 * nn], pa, b0, b1);
+      mma_bf16_16816(o_acc[2 * nn + 1], pa, b2, b3);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+
+  // -------------------------------------------------- merge the four warps
+  // every consumer reached here; the ring is idle (all issued tiles consumed)
+  asm volatile("bar.sync 1, %0;" ::"n"(C::kConsumerWarps * 32) : "memory");
+  if (aborted || *reinterpret_cast<volatile int*>(abort_flag)) {
+    // a wait gave up: leave the partial as NaN so the result is visibly invalid
+    const size_t item = ((size_t)b * p.Hkv + g) * p.max_chunks + c;
+    for (int r = threadIdx.x; r < p.R; r += C::kConsumerWarps * 32) p.part_lse[item * p.R + r] = NAN;
+    return;
+  }
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+  float* st = stats + ((mt * 4 + wsub) * 16) * 2;
+  if (tig == 0) {
+    st[gid * 2 + 0] = m0;
+    st[gid * 2 + 1] = l0;
+    st[(gid + 8) * 2 + 0] = m1;
+    st[(gid + 8) * 2 + 1] = l1;
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(C::kConsumerWarps * 32) : "memory");
+  float M0 = -INFINITY, M1 = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const float* sw = stats + ((mt * 4 + w) * 16) * 2;
+    M0 = fmaxf(M0, sw[gid * 2]);
+    M1 = fmaxf(M1, sw[(gid + 8) * 2]);
+  }
+  const float f0 = (m0 == -INFINITY) ? 0.f : ex2(m0 - M0);
+  const float f1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - M1);
+  float* red = reinterpret_cast<float*>(smem) + ((mt * 4 + wsub) * 16) * C::kRedStride;
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) {
+    const int col = n * 8 + tig * 2;
+    *reinterpret_cast<float2*>(red + gid * C::kRedStride + col) = make_float2(o_acc[n][0] * f0, o_acc[n][1] * f0);
+    *reinterpret_cast<float2*>(red + (gid + 8) * C::kRedStride + col) =
+        make_float2(o_acc[n][2] * f1, o_acc[n][3] * f1);
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(C::kConsumerWarps * 32) : "memory");
+
+  const size_t item = ((size_t)b * p.Hkv + g) * p.max_chunks + c;
+  float* out = p.part_o + item * (size_t)p.R * D;
+  constexpr int kVec = D / 4;   // float4 per row
+  for (int idx = threadIdx.x; idx < p.R * kVec; idx += C::kConsumerWarps * 32) {
+    const int r = idx / kVec, col = (idx - r * kVec) * 4;
+    const int rm = r >> 4, rr = r & 15;
+    float mrow = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) mrow = fmaxf(mrow, stats[((rm * 4 + w) * 16 + rr) * 2]);
+    float lsum = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float mw = stats[((rm * 4 + w) * 16 + rr) * 2];
+      const float fw = (mw == -INFINITY) ? 0.f : ex2(mw - mrow);
+      lsum += stats[((rm * 4 + w) * 16 + rr) * 2 + 1] * fw;
+      const float4 x = *reinterpret_cast<const float4*>(reinterpret_cast<float*>(smem) +
+                                                        ((rm * 4 + w) * 16 + rr) * C::kRedStride + col);
+      acc.x += x.x;
+      acc.y += x.y;
+      acc.z += x.z;
+      acc.w += x.w;
+    }
+    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+    *reinterpret_cast<float4*>(out + (size_t)r * D + col) =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    if (col == 0) p.part_lse[item * p.R + r] = lsum > 0.f ? (mrow + log2f(lsum)) * kLn2 : -INFINITY;
+  }
+}
+
+// One warp per output row (b, t, h): merge the chunk partials of that row.
+template <int D>
+__global__ void __launch_bounds__(256) decode_combine_kernel(const float* __restrict__ part_o,
+                                                             const float* __restrict__ part_lse,
+                                                             const int32_t* __restrict__ seqlens, void* o, int o_bf16,
+                                                             float* lse, SplitParams p, int B, int paged) {
+  const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int rows = B * p.T * p.Hq;
+  if (warp_global >= rows) return;
+  const int h = warp_global % p.Hq;
+  const int t = (warp_global / p.Hq) % p.T;
+  const int b = warp_global / (p.Hq * p.T);
+  const int g = h / p.G, r = t * p.G + (h - g * p.G);
+  constexpr int kPer = D / 32;   // output columns per lane
+  float acc[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+  float lse_row;
+
+  const int L = seqlens[b];
+  if (seqlen_bad(L, p.T, p.max_seqlen, paged != 0, p.capacity, p.max_blocks)) {
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) acc[e] = NAN;
+    lse_row = NAN;
+  } else {
+    const int nc = (L + p.chunk - 1) / p.chunk;
+    const size_t item0 = ((size_t)b * p.Hkv + g) * p.max_chunks;
+    float M = -INFINITY;
+    for (int c = lane; c < nc; c += 32) M = fmaxf(M, part_lse[(item0 + c) * p.R + r]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float z = 0.f;
+    for (int c = lane; c < nc; c += 32) {
+      const float lc = part_lse[(item0 + c) * p.R + r];
+      z += (lc == -INFINITY) ? 0.f : expf(lc - M);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+    lse_row = M + logf(z);
+    for (int c = 0; c < nc; ++c) {
+      const float lc = part_lse[(item0 + c) * p.R + r];
+      if (lc == -INFINITY) continue;
+      const float w = expf(lc - lse_row);
+      const float* src = part_o + ((item0 + c) * p.R + r) * D + lane * kPer;
+      if constexpr (kPer == 4) {
+        const float4 x = *reinterpret_cast<const float4*>(src);
+        acc[0] += w * x.x;
+        acc[1] += w * x.y;
+        acc[2] += w * x.z;
+        acc[3] += w * x.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) acc[e] += w * src[e];
+      }
+    }
+  }
+  const size_t orow = (((size_t)b * p.T + t) * p.Hq + h) * D + lane * kPer;
+  if (o_bf16) {
+    __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(o) + orow;
+#pragma unroll
+    for (int e = 0; e < kPer; e += 2) *reinterpret_cast<__nv_bfloat162*>(ob + e) = __floats2bfloat162_rn(acc[e], acc[e + 1]);
+  } else {
+    float* of = reinterpret_cast<float*>(o) + orow;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) of[e] = acc[e];
+  }
+  if (lse && lane == 0) lse[((size_t)b * p.Hq + h) * p.T + t] = lse_row;
+}
+
+template <int D, int MT, bool PAGED>
+cudaError_t run_split(const CUtensorMap& tk, const CUtensorMap& tv, const SplitParams& sp, int B,
+                      cudaStream_t stream) {
+  using C = DecodeCfg<D, MT>;
+  auto kern = decode_split_kernel<D, MT, PAGED>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid(sp.max_chunks, sp.Hkv, B);
+  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(tk, tv, sp);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int decode_chunk_tokens(int B, int Hkv, int rows, int max_seqlen, int num_splits) {
+  int chunk;
+  if (num_splits > 0) {
+    chunk = (max_seqlen + num_splits - 1) / num_splits;
+  } else {
+    chunk = rows <= 8 ? 512 : (rows <= 16 ? 1024 : 2048);
+    // short caches: keep at least ~2 work items per SM
+    while (chunk > 256 && (long long)B * Hkv * ((max_seqlen + chunk - 1) / chunk) < 296) chunk >>= 1;
+  }
+  chunk = ((chunk + kDecodeTile - 1) / kDecodeTile) * kDecodeTile;
+  return chunk < kDecodeTile ? kDecodeTile : chunk;
+}
+
+cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
+  const bool paged = a.page_table != nullptr;
+  const int G = a.Hq / a.Hkv, R = G * a.T;
+  SplitParams sp;
+  sp.q = static_cast<const __nv_bfloat16*>(a.q);
+  sp.seqlens = a.seqlens;
+  sp.page_table = a.page_table;
+  sp.part_o = a.part_o;
+  sp.part_lse = a.part_lse;
+  sp.status = a.status;
+  sp.T = a.T;
+  sp.Hq = a.Hq;
+  sp.Hkv = a.Hkv;
+  sp.G = G;
+  sp.R = R;
+  sp.chunk = a.chunk;
+  sp.max_chunks = a.max_chunks;
+  sp.capacity = a.capacity;
+  sp.max_blocks = a.max_blocks;
+  sp.num_blocks = a.num_blocks;
+  sp.max_seqlen = a.max_seqlen;
+  sp.scale_log2 = a.scale * kLog2e;
+  sp.causal = a.causal;
+
+  // K/V viewed as 3-D {d, Hkv, rows}: rows = B * capacity (contiguous) or num_blocks * 16 (paged)
+  const uint64_t rows = paged ? (uint64_t)a.num_blocks * kPageTokens : (uint64_t)a.B * a.capacity;
+  const uint32_t box_rows = paged ? kPageTokens : kDecodeTile;
+  CUtensorMap tk, tv;
+  const uint64_t s1 = (uint64_t)a.d * 2, s2 = (uint64_t)a.Hkv * a.d * 2;
+  if (encode_tmap_3d(&tk, a.k, a.d, a.Hkv, rows, s1, s2, 64, 1, box_rows) ||
+      encode_tmap_3d(&tv, a.v, a.d, a.Hkv, rows, s1, s2, 64, 1, box_rows))
+    return cudaErrorInvalidValue;
+
+  cudaError_t e;
+  if (a.d == 128) {
+    if (R <= 16) e = paged ? run_split<128, 1, true>(tk, tv, sp, a.B, stream) : run_split<128, 1, false>(tk, tv, sp, a.B, stream);
+    else e = paged ? run_split<128, 2, true>(tk, tv, sp, a.B, stream) : run_split<128, 2, false>(tk, tv, sp, a.B, stream);
+  } else {
+    if (R <= 16) e = paged ? run_split<64, 1, true>(tk, tv, sp, a.B, stream) : run_split<64, 1, false>(tk, tv, sp, a.B, stream);
+    else e = paged ? run_split<64, 2, true>(tk, tv, sp, a.B, stream) : run_split<64, 2, false>(tk, tv, sp, a.B, stream);
+  }
+  if (e != cudaSuccess) return e;
+
+  const int rows_out = a.B * a.T * a.Hq;
+  const int blocks = (rows_out * 32 + 255) / 256;
+  if (a.d == 128)
+    decode_combine_kernel<128><<<blocks, 256, 0, stream>>>(a.part_o, a.part_lse, a.seqlens, a.o, a.o_bf16, a.lse, sp,
+                                                           a.B, paged ? 1 : 0);
+  else
+    decode_combine_kernel<64><<<blocks, 256, 0, stream>>>(a.part_o, a.part_lse, a.seqlens, a.o, a.o_bf16, a.lse, sp,
+                                                          a.B, paged ? 1 : 0);
+  return cudaGetLastError();
+}
+
+}  // namespace kvattn

@@ -1,0 +1,76 @@
+// Launchers shared between the C-ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace kvattn {
+
+constexpr int kPageTokens = 16;   // tokens per physical KV block
+constexpr int kDecodeTile = 64;   // tokens per pipeline stage of the decode kernel
+
+struct DecodeLaunch {
+  const void* q;
+  const void* k;          // contiguous cache or paged pool
+  const void* v;
+  const int32_t* seqlens;
+  const int32_t* page_table;  // nullptr = contiguous
+  int max_blocks, num_blocks, capacity, max_seqlen;
+  void* o;
+  int o_bf16;
+  float* lse;
+  int B, T, Hq, Hkv, d;
+  float scale;
+  int causal;
+  int chunk;          // tokens per split (multiple of kDecodeTile)
+  int max_chunks;     // ceil(max_seqlen / chunk)
+  float* part_o;      // [B, Hkv, max_chunks, R, d]
+  float* part_lse;    // [B, Hkv, max_chunks, R]
+  unsigned* status;
+};
+
+struct PrefillLaunch {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  int o_bf16;
+  float* lse;
+  int B, Hq, Hkv, N, d;
+  float scale;
+  int causal;
+  unsigned* status;
+};
+
+struct AppendLaunch {
+  void* k;
+  void* v;
+  const void* k_new;
+  const void* v_new;
+  const int32_t* cache_lens;
+  const int32_t* page_table;
+  int max_blocks, num_blocks, capacity;
+  int B, T, Hkv, d;
+  unsigned* status;
+};
+
+// Tokens per split for attn_decode (host heuristic, deterministic in its inputs).
+int decode_chunk_tokens(int B, int Hkv, int rows, int max_seqlen, int num_splits);
+
+// Encode a rank-N (1..5) bf16 tiled tensor map with 128-byte swizzle; strides
+// in bytes for dims 1..N-1.  Returns 0 on success.
+int encode_tmap_nd(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
+                   const cuuint64_t* strides_bytes, const cuuint32_t* box);
+
+// Encode a 3-D bf16 tiled tensor map {inner, mid, rows} with 128-byte swizzle.
+// Strides are in bytes for dims 1 and 2.  Returns 0 on success.
+int encode_tmap_3d(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2,
+                   uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1, uint32_t box2);
+
+cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream);
+cudaError_t launch_append(const AppendLaunch& a, cudaStream_t stream);
+cudaError_t launch_prefill(const PrefillLaunch& a, cudaStream_t stream);
+
+}  // namespace kvattn
