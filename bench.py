@@ -1,0 +1,565 @@
+"""Benchmark: prefill attention TFLOP/s and KV-cache decode GB/s on B200.
+
+One step is one pass of the whole hot path on the Llama-3.1-8B attention-layer
+shapes (Hq=32, Hkv=8, d=128, bf16 in, fp32 accumulation):
+
+* causal prefill, B=4, N=4096 (attn_prefill, tcgen05 kernel);
+* a decode step for B=16 sequences whose cache lengths are uniform in
+  [1024, 32768]: kv_append of one new token per sequence, then split-KV
+  attn_decode (split kernel + log-sum-exp combine) against the contiguous cache.
+
+``value`` is the prefill throughput in TFLOP/s (algorithmic FLOPs: 4 d per
+visible query-key pair, masked work not credited) over the prefill kernel's own
+device time; the ``decode`` object gives the KV-cache GB/s (algorithmic bytes:
+every valid K and V byte plus q, o, lse and lengths) over the attn_decode
+device time.  Both are whole-job figures: summed over ranks, divided by the
+slowest rank's time.  Inputs (192 MiB prefill, 1 GB cache) exceed the 126 MB
+L2, so no explicit flush is needed.
+
+``--impl reference`` times the fp64 CPU oracle on bounded samples of the same
+workload instead (rank 0 only).  ``--workload`` selects another shape set for
+manual runs; the default is the one described above.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "prefill attention TFLOP/s and decode KV-cache GB/s, % of B200 roofline"
+
+# prefill workload / decode workload pairs (names from synth.WORKLOADS)
+WORKLOAD_SETS = {
+    "llama8b_layer": ("prefill_llama8b", "decode_contig"),
+    "gpt2_prefill_paged_decode": ("prefill_gpt2", "decode_paged"),
+    "llama8b_nc_paged_t4": ("prefill_llama8b_nc", "decode_paged_t4"),
+}
+DEFAULT_SET = "llama8b_layer"
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in PEAKS_FALLBACK}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ----------------------------------------------------------------- ranks
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        from datetime import timedelta
+        dist.init_process_group(backend=backend, timeout=timedelta(seconds=120))
+    return dist
+
+
+def reduce_over_ranks(local_sum: float, local_max: float, world: int, device=None):
+    """(sum over ranks of local_sum, max over ranks of local_max)."""
+    if world == 1:
+        return local_sum, local_max
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([local_sum], dtype=torch.float64, device=device)
+    m = torch.tensor([local_max], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    dist.all_reduce(m, op=dist.ReduceOp.MAX)
+    return float(t.item()), float(m.item())
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples, kept only inside [t0, t1]."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.rows = []
+        self.window = (0.0, 0.0)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        t0, t1 = self.window
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ts, line in self.rows:
+            if not (t0 - 0.05 <= ts <= t1 + 0.05):
+                continue
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                sm.append(float(parts[2]))
+                smax.append(float(parts[3]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[6:10]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- workload
+def decode_bytes(case, w) -> int:
+    """Algorithmic bytes of one attn_decode call: valid K and V, q, o (bf16), lse, lengths (+ page table)."""
+    kvb = int(case.seqlens_k.sum()) * w.Hkv * w.d * 2 * 2
+    qo = 2 * w.B * w.T * w.Hq * w.d * 2
+    lse = w.B * w.Hq * w.T * 4
+    lens = w.B * 4
+    table = 0
+    if case.paged:
+        table = int(sum((int(L) + 15) // 16 for L in case.seqlens_k)) * 4
+    return kvb + qo + lse + lens + table
+
+
+def prefill_flops(w) -> int:
+    pairs = w.N * (w.N + 1) // 2 if w.causal else w.N * w.N
+    return 4 * w.B * w.Hq * w.d * pairs
+
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    import kv_cache_decode_attn_b200 as kv
+    import synth
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    pf_name, dec_name = WORKLOAD_SETS[args.workload]
+    wp = synth.WORKLOADS[pf_name]
+    wd = synth.WORKLOADS[dec_name]
+    seed_off = 7919 * rank   # weak scaling: every rank gets its own batch
+    q, k, v = synth.prefill_inputs(wp.B, wp.Hq, wp.Hkv, wp.N, wp.d, synth.SEEDS[pf_name] + seed_off, dev)
+    o = torch.empty(wp.B, wp.N, wp.Hq, wp.d, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(wp.B, wp.Hq, wp.N, dtype=torch.float32, device=dev)
+    case = synth.decode_inputs(wd.B, wd.T, wd.Hq, wd.Hkv, wd.d, wd.len_lo, wd.len_hi,
+                               synth.SEEDS[dec_name] + seed_off, device=dev, paged=wd.paged)
+    cache_lens = torch.as_tensor(case.cache_lens.astype(np.int32), device=dev)
+    seqlens = torch.as_tensor(case.seqlens_k.astype(np.int32), device=dev)
+    table = None if case.page_table is None else torch.as_tensor(case.page_table, device=dev)
+    kc = case.k_pool if wd.paged else case.k_cache
+    vc = case.v_pool if wd.paged else case.v_cache
+    msk = int(case.seqlens_k.max())
+    od = torch.empty(wd.B, wd.T, wd.Hq, wd.d, dtype=torch.bfloat16, device=dev)
+    ld = torch.empty(wd.B, wd.Hq, wd.T, dtype=torch.float32, device=dev)
+    ws = kv.decode_workspace(wd.B, wd.T, wd.Hq, wd.Hkv, wd.d, msk, 0, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        kv.attn_prefill(q, k, v, o, lse, scale=wp.scale, causal=wp.causal, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        # the same token position is appended every step, so the cache length stays fixed
+        kv.kv_append(kc, vc, case.k_new, case.v_new, cache_lens, page_table=table, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        kv.attn_decode(case.q, kc, vc, seqlens, od, ld, page_table=table, max_seqlen_k=msk, scale=wd.scale,
+                       causal=wd.causal, workspace=ws, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    kv.attn_get_device_status(clear=True)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    wall0 = time.time()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(events[i])
+    t_stop.record(stream)
+    torch.cuda.synchronize(dev)
+    wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    clocks.window = (wall0, wall1)
+    time.sleep(0.25)
+    clocks.stop()
+    status = kv.attn_get_device_status(clear=True)
+    if status != 0:
+        raise RuntimeError(f"device status {status} during the benchmark")
+
+    total_ms = t_start.elapsed_time(t_stop)
+    pf_ms = sum(e[0].elapsed_time(e[1]) for e in events)
+    ap_ms = sum(e[1].elapsed_time(e[2]) for e in events)
+    dec_ms = sum(e[2].elapsed_time(e[3]) for e in events)
+    K = args.steps
+    flops = prefill_flops(wp)
+    dbytes = decode_bytes(case, wd)
+
+    # whole-job: units summed over ranks / slowest rank's time
+    tot_flops, pf_max = reduce_over_ranks(flops * K, pf_ms, world, dev)
+    tot_bytes, dec_max = reduce_over_ranks(dbytes * K, dec_ms, world, dev)
+    _, total_max = reduce_over_ranks(0.0, total_ms, world, dev)
+    pf_tflops = tot_flops / (pf_max * 1e-3) / 1e12
+    dec_gbs = tot_bytes / (dec_max * 1e-3) / 1e9
+
+    # -------- end to end through the public API with host buffers (pinned)
+    e2e = None if args.no_e2e else run_e2e(kv, torch, dev, stream, wp, wd, q, k, v, case, table, msk, ws, args,
+                                           world)
+
+    peaks, peak_src = load_peaks()
+    pf_kernel_tflops = flops / (pf_ms / K * 1e-3) / 1e12          # per launch, this rank
+    dec_kernel_gbs = dbytes / (dec_ms / K * 1e-3) / 1e9
+    traffic = load_traffic()
+    roof_pf = {"bound": "tensor", "achieved": round(pf_kernel_tflops, 1), "peak": peaks["bf16_tflops"],
+               "unit": "TFLOP/s", "frac": round(pf_kernel_tflops / peaks["bf16_tflops"], 4),
+               "frac_of_sustained": round(pf_kernel_tflops / peaks["bf16_tflops_sustained"], 4),
+               "peak_source": f"{peak_src} (bf16 burst)", "traffic": traffic.get("prefill"),
+               "kernel": "prefill_kernel<128>", "flops_per_launch": flops,
+               "launch_ms": round(pf_ms / K, 4)}
+    roof_dec = {"bound": "hbm", "achieved": round(dec_kernel_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(dec_kernel_gbs / peaks["hbm_gbs"], 4), "peak_source": f"{peak_src} (copy)",
+                "traffic": traffic.get("decode"), "kernel": "decode_split_kernel + decode_combine_kernel",
+                "bytes_per_launch": dbytes, "launch_ms": round(dec_ms / K, 4)}
+
+    out = None
+    if rank == 0:
+        cpu = cpu_baseline(args, wp, wd, q, k, v, case) if (world == 1 and not args.no_cpu_baseline) else None
+        out = {
+            "metric": METRIC, "value": round(pf_tflops, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": round(total_max / K, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {
+                "workload": args.workload,
+                "prefill": {"name": pf_name, "B": wp.B, "Hq": wp.Hq, "Hkv": wp.Hkv, "N": wp.N, "d": wp.d,
+                            "causal": wp.causal, "o_dtype": "bf16"},
+                "decode": {"name": dec_name, "B": wd.B, "T": wd.T, "Hq": wd.Hq, "Hkv": wd.Hkv, "d": wd.d,
+                           "cache_len": [wd.len_lo, wd.len_hi], "paged": wd.paged, "append_before_attend": True,
+                           "kv_bytes_per_step": int(case.seqlens_k.sum()) * wd.Hkv * wd.d * 4},
+                "l2": "no flush: every step reads inputs larger than the 126 MB L2",
+                "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                "seed": synth.SEEDS[pf_name],
+            },
+            "decode": {"value": round(dec_gbs, 1), "unit": "GB/s", "roofline": roof_dec,
+                       "append_ms_per_step": round(ap_ms / K, 4)},
+            "roofline": roof_pf,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 4 * K,   # prefill, append, decode split, decode combine per step
+            "clocks": clocks.summary(),
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return out
+
+
+def run_e2e(kv, torch, dev, stream, wp, wd, q, k, v, case, table, msk, ws, args, world):
+    """Same step through the public API, inputs copied from pinned host memory
+    and results read back every step (the KV cache stays resident: it is state)."""
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    ho = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    hl = torch.empty(wp.B, wp.Hq, wp.N, dtype=torch.float32).pin_memory()
+    hdq, hkn, hvn = (t.cpu().pin_memory() for t in (case.q, case.k_new, case.v_new))
+    hcl = torch.as_tensor(case.cache_lens.astype(np.int32)).pin_memory()
+    hsl = torch.as_tensor(case.seqlens_k.astype(np.int32)).pin_memory()
+    hdo = torch.empty(case.q.shape, dtype=torch.bfloat16).pin_memory()
+    hdl = torch.empty(wd.B, wd.Hq, wd.T, dtype=torch.float32).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    do = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    dl = torch.empty(wp.B, wp.Hq, wp.N, dtype=torch.float32, device=dev)
+    ddq, dkn, dvn = torch.empty_like(case.q), torch.empty_like(case.k_new), torch.empty_like(case.v_new)
+    dcl = torch.empty(wd.B, dtype=torch.int32, device=dev)
+    dsl = torch.empty(wd.B, dtype=torch.int32, device=dev)
+    ddo = torch.empty(case.q.shape, dtype=torch.bfloat16, device=dev)
+    ddl = torch.empty(wd.B, wd.Hq, wd.T, dtype=torch.float32, device=dev)
+    kc = case.k_pool if wd.paged else case.k_cache
+    vc = case.v_pool if wd.paged else case.v_cache
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        kv.attn_prefill(dq, dk, dv, do, dl, scale=wp.scale, causal=wp.causal, stream=stream)
+        ho.copy_(do, non_blocking=True)
+        hl.copy_(dl, non_blocking=True)
+        if ev is not None:
+            ev[1].record(stream)
+        ddq.copy_(hdq, non_blocking=True)
+        dkn.copy_(hkn, non_blocking=True)
+        dvn.copy_(hvn, non_blocking=True)
+        dcl.copy_(hcl, non_blocking=True)
+        dsl.copy_(hsl, non_blocking=True)
+        kv.kv_append(kc, vc, dkn, dvn, dcl, page_table=table, stream=stream)
+        kv.attn_decode(ddq, kc, vc, dsl, ddo, ddl, page_table=table, max_seqlen_k=msk, scale=wd.scale,
+                       causal=wd.causal, workspace=ws, stream=stream)
+        hdo.copy_(ddo, non_blocking=True)
+        hdl.copy_(ddl, non_blocking=True)
+        if ev is not None:
+            ev[2].record(stream)
+
+    n = max(3, min(args.steps, 20))
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+    for i in range(n):
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    pf_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    dec_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    flops, pf_max = reduce_over_ranks(prefill_flops(wp) * n, pf_ms, world, dev)
+    dbytes, dec_max = reduce_over_ranks(decode_bytes(case, wd) * n, dec_ms, world, dev)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdq, hkn, hvn, hcl, hsl))
+    d2h = sum(t.numel() * t.element_size() for t in (ho, hl, hdo, hdl))
+    return {"value": round(flops / (pf_max * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": n,
+            "decode": {"value": round(dbytes / (dec_max * 1e-3) / 1e9, 1), "unit": "GB/s"}}
+
+
+def load_traffic():
+    """Per-launch DRAM bytes from the committed ncu summary, if it matches the current kernels."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            return json.load(f)
+    except (OSError, ValueError):
+        return {}
+
+
+# ------------------------------------------------------------ CPU oracle legs
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        if info:
+            return int(max(i.get("num_threads", 1) for i in info))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+ORACLE_ROWS = 256   # query rows per oracle prefill sample
+
+
+def oracle_prefill_sample(wp, q, k, v, budget_s, rng):
+    """Blocks of 256 query rows of one (b, h) head through the oracle until the
+    budget is spent.  q, k, v are host bf16 tensors; each block's slices are
+    converted to float64 before its clock starts."""
+    import oracle
+    flops, t, blocks = 0, 0.0, 0
+    G = wp.Hq // wp.Hkv
+    while True:
+        b, h = int(rng.integers(wp.B)), int(rng.integers(wp.Hq))
+        i0 = int(rng.integers(0, max(1, wp.N - ORACLE_ROWS + 1)))
+        i1 = min(wp.N, i0 + ORACLE_ROWS)
+        nk = i1 if wp.causal else wp.N      # rows i0..i1-1 are the last rows of the first i1 keys
+        g = h // G
+        qs = q[b, i0:i1, h].double().numpy()
+        ks = k[b, :nk, g].double().numpy()
+        vs = v[b, :nk, g].double().numpy()
+        t0 = time.perf_counter()
+        oracle.attend_head(qs, ks, vs, wp.scale, wp.causal)
+        t += time.perf_counter() - t0
+        flops += 4 * wp.d * oracle.visible_pairs(i1 - i0, nk, wp.causal)
+        blocks += 1
+        if t >= budget_s:
+            return flops, t, blocks
+
+
+def oracle_decode_sample(wd, case_h, budget_s, rng):
+    """One KV head group of one sequence (its Hq/Hkv query heads, all T tokens)
+    through the oracle per sample, until the budget is spent."""
+    import oracle
+    nbytes, t, units = 0, 0.0, 0
+    G = wd.Hq // wd.Hkv
+    while True:
+        b = int(rng.integers(case_h["q"].shape[0]))
+        g = int(rng.integers(wd.Hkv))
+        L = int(case_h["seqlens_k"][b])
+        qs = case_h["q"][b:b + 1, :, g * G:(g + 1) * G]
+        kc, vc = case_h["k"][b:b + 1, :L, g:g + 1], case_h["v"][b:b + 1, :L, g:g + 1]
+        t0 = time.perf_counter()
+        oracle.decode(qs, kc, vc, [L], wd.scale, wd.causal)
+        t += time.perf_counter() - t0
+        nbytes += L * wd.d * 4 + 2 * wd.T * G * wd.d * 2
+        units += 1
+        if t >= budget_s:
+            return nbytes, t, units
+
+
+def host_decode_case(case, wd, max_seqs=4):
+    """fp64 host copies of a few sequences of the decode workload (cache as it is
+    after the append: stored rows followed by the new tokens)."""
+    import torch
+    idx = list(range(min(max_seqs, wd.B)))
+    Lmax = int(max(case.seqlens_k[i] for i in idx))
+    k = np.zeros((len(idx), Lmax, wd.Hkv, wd.d))
+    v = np.zeros_like(k)
+    for j, b in enumerate(idx):
+        L0 = int(case.cache_lens[b])
+        if case.paged:
+            nb = (L0 + wd.T + 15) // 16
+            ids = torch.as_tensor(case.page_table[b, :nb].astype(np.int64), device=case.k_pool.device)
+            kb = case.k_pool.index_select(0, ids).reshape(nb * 16, wd.Hkv, wd.d)[:L0]
+            vb = case.v_pool.index_select(0, ids).reshape(nb * 16, wd.Hkv, wd.d)[:L0]
+        else:
+            kb, vb = case.k_cache[b, :L0], case.v_cache[b, :L0]
+        k[j, :L0] = kb.float().cpu().numpy()
+        v[j, :L0] = vb.float().cpu().numpy()
+        k[j, L0:L0 + wd.T] = case.k_new[b].float().cpu().numpy()
+        v[j, L0:L0 + wd.T] = case.v_new[b].float().cpu().numpy()
+    return {"q": case.q[idx].float().cpu().numpy().astype(np.float64), "k": k, "v": v,
+            "seqlens_k": case.seqlens_k[idx]}
+
+
+def cpu_baseline(args, wp, wd, q, k, v, case):
+    rng = np.random.default_rng(0)
+    qh, kh, vh = (t.cpu() for t in (q, k, v))
+    fl, tp, blocks = oracle_prefill_sample(wp, qh, kh, vh, args.cpu_budget, rng)
+    ch = host_decode_case(case, wd)
+    nb, td, units = oracle_decode_sample(wd, ch, args.cpu_budget / 2, rng)
+    return {"value": round(fl / tp / 1e12, 5), "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
+            "sample": f"{blocks} blocks of {ORACLE_ROWS} query rows of single (b, h) heads of the prefill "
+                      f"workload ({tp:.1f} s); decode: {units} (sequence, KV head) groups with all their "
+                      f"query heads ({td:.1f} s)",
+            "decode": {"value": round(nb / td / 1e9, 4), "unit": "GB/s"}}
+
+
+def run_reference(args):
+    """The oracle, as it stands, on the host cores: bounded samples of the same workload per step."""
+    import synth
+    pf_name, dec_name = WORKLOAD_SETS[args.workload]
+    wp, wd = synth.WORKLOADS[pf_name], synth.WORKLOADS[dec_name]
+    q, k, v = synth.prefill_inputs(wp.B, wp.Hq, wp.Hkv, wp.N, wp.d, synth.SEEDS[pf_name], "cpu")
+    n_seq = 2   # sequences of the decode workload held on the host for sampling
+    case = synth.decode_inputs(n_seq, wd.T, wd.Hq, wd.Hkv, wd.d, wd.len_lo, wd.len_hi, synth.SEEDS[dec_name],
+                               device="cpu", paged=wd.paged)
+    ch = host_decode_case(case, _shrink(wd, n_seq), max_seqs=n_seq)
+    rng = np.random.default_rng(1)
+    # each step is a bounded sample, sized so the whole run stays within a few minutes
+    per_step = min(args.ref_step_budget, 150.0 / (args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_prefill_sample(wp, q, k, v, per_step * 0.7, rng)
+    fl_tot = t_pf = nb_tot = t_dec = 0.0
+    blocks = units = 0
+    for _ in range(args.steps):
+        fl, tp, nbk = oracle_prefill_sample(wp, q, k, v, per_step * 0.7, rng)
+        nb, td, nu = oracle_decode_sample(wd, ch, per_step * 0.3, rng)
+        fl_tot += fl
+        t_pf += tp
+        blocks += nbk
+        nb_tot += nb
+        t_dec += td
+        units += nu
+    value = fl_tot / t_pf / 1e12
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round((t_pf + t_dec) / args.steps * 1e3, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "prefill": pf_name, "decode": dec_name,
+                   "sample": f"each step: blocks of {ORACLE_ROWS} prefill query rows for ~70% and (sequence, KV "
+                             f"head) decode groups for ~30% of a {per_step:.3f} s budget"},
+        "decode": {"value": round(nb_tot / t_dec / 1e9, 5), "unit": "GB/s"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
+                         "sample": f"{blocks} prefill row blocks, {units} decode groups over {args.steps} steps"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def _shrink(wd, B):
+    import dataclasses
+    return dataclasses.replace(wd, B=B)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOAD_SETS), default=DEFAULT_SET)
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--ref-step-budget", type=float, default=1.5, help="seconds of oracle work per reference step")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args)), flush=True)
+        return 0
+    if world != args.gpus and world > 1:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    out = run_ours(args, world, rank, local)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
