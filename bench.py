@@ -379,13 +379,26 @@ def run_e2e(kv, torch, dev, stream, wp, wd, q, k, v, case, table, msk, ws, args,
 
 
 def load_traffic():
-    """Per-launch DRAM bytes from the committed ncu summary, if it matches the current kernels."""
+    """Per-launch DRAM bytes (ncu dram__bytes_read + dram__bytes_write) from the
+    committed profile summary, kept only while the kernel source it was measured
+    on is unchanged (first 16 hex digits of its sha256)."""
+    import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            return json.load(f)
+            d = json.load(f)
     except (OSError, ValueError):
         return {}
+    out = {}
+    for key, src in (("prefill", "prefill.cu"), ("decode", "decode.cu")):
+        try:
+            with open(os.path.join(ROOT, "kv_cache_decode_attn_b200", "csrc", src), "rb") as f:
+                h = hashlib.sha256(f.read()).hexdigest()[:16]
+        except OSError:
+            continue
+        if d.get(f"{key}_source_sha256_16") == h and key in d:
+            out[key] = d[key]
+    return out
 
 
 # ------------------------------------------------------------ CPU oracle legs
