@@ -180,6 +180,42 @@ ATTN_API int64_t kv_cache_bytes(int n_layers, int batch, int64_t tokens, int n_k
  */
 ATTN_API int attn_get_device_status(int clear);
 
+/*
+ * attn_decode_noalloc -- attn_decode for callers that cannot allocate device
+ * memory.  The pages have no counterpart: this is a packaging variant only.
+ *
+ * Some callers have no way to hand the library a workspace: a plugin loaded by
+ * a host program that passes it nothing but input and output pointers, or a
+ * serving process that reserves every byte of device memory at start-up for
+ * weights and its KV pool and treats any later cudaMalloc (which can also
+ * synchronise the device) as an error.  This entry point takes exactly the
+ * arguments of attn_decode except the workspace, and computes the same result
+ * with the same kernels.  The per-chunk partials live in one file-scope device
+ * array of ATTN_DECODE_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads
+ * the library keeps from the first call on that device until the process
+ * exits.  Nothing here calls cudaMalloc, cudaFree or an allocating library
+ * routine.
+ *
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture on the device.
+ *   - All calls share the one array and leave the last call's partials in it.
+ *     Nothing in it has to start at zero (every partial is written before it is
+ *     read), but calls whose kernels overlap on the GPU -- on different streams,
+ *     or from different host threads -- race on it: serialise them.
+ *   - Returns ATTN_ERR_WORKSPACE, before launching anything, when the request
+ *     needs more than ATTN_DECODE_NOALLOC_SCRATCH_BYTES of partials (the figure
+ *     attn_decode_workspace_bytes reports); a smaller num_splits needs less.
+ *     Every other error is attn_decode's.
+ */
+#define ATTN_DECODE_NOALLOC_SCRATCH_BYTES (32u << 20) /* 32 MiB */
+
+ATTN_API int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens_k,
+                                 const int32_t* page_table, int max_blocks_per_seq, int num_blocks,
+                                 int cache_capacity, int max_seqlen_k, void* o, int o_dtype, float* lse, int B,
+                                 int T, int Hq, int Hkv, int d, float scale, int causal, int num_splits,
+                                 void* stream);
+
 /* attn_status_string -- static text for a return code (never NULL). */
 ATTN_API const char* attn_status_string(int status);
 

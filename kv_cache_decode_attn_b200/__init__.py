@@ -20,7 +20,8 @@ import torch
 
 __all__ = [
     "lib", "LIB_PATH", "AttnError",
-    "attn_prefill", "attn_decode", "attn_decode_workspace_bytes", "kv_append", "kv_cache_bytes",
+    "attn_prefill", "attn_decode", "attn_decode_workspace_bytes", "attn_decode_noalloc", "kv_append",
+    "kv_cache_bytes", "ATTN_DECODE_NOALLOC_SCRATCH_BYTES",
     "attn_get_device_status", "attn_status_string", "decode_workspace",
     "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_WORKSPACE", "ATTN_ERR_CUDA",
     "ATTN_ERR_DEVICE", "ATTN_F32", "ATTN_BF16", "ATTN_DEV_PAGE_ID", "ATTN_DEV_SEQLEN",
@@ -31,6 +32,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvattn.s
 
 ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_WORKSPACE, ATTN_ERR_CUDA, ATTN_ERR_DEVICE = 0, -1, -2, -3, -4, -5
 ATTN_F32, ATTN_BF16 = 0, 1
+ATTN_DECODE_NOALLOC_SCRATCH_BYTES = 32 << 20
 ATTN_DEV_PAGE_ID, ATTN_DEV_SEQLEN, ATTN_DEV_APPEND_RANGE, ATTN_DEV_TIMEOUT = 1, 2, 4, 8
 
 _p, _i, _i64, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
@@ -40,6 +42,8 @@ _SIGNATURES = {
     "attn_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "attn_decode": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _p, _i, _p, _i, _i, _i, _i, _i, _f, _i, _i, _p, _sz,
                          _p]),
+    "attn_decode_noalloc": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _p, _i, _p, _i, _i, _i, _i, _i, _f, _i, _i,
+                                 _p]),
     "kv_append": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p]),
     "kv_cache_bytes": (_i64, [_i, _i, _i64, _i, _i, _i]),
     "attn_get_device_status": (_i, [_i]),
@@ -156,6 +160,27 @@ def attn_decode(q, k_cache, v_cache, seqlens_k, o, lse=None, page_table=None, ma
                          int(bool(causal)), int(num_splits), _dev(workspace, "workspace"),
                          workspace.numel() * workspace.element_size(), _stream(stream))
     _check("attn_decode", st)
+
+
+def attn_decode_noalloc(q, k_cache, v_cache, seqlens_k, o, lse=None, page_table=None, max_seqlen_k=0, scale=None,
+                        causal=True, num_splits=0, stream=None) -> None:
+    """``attn_decode`` for callers that cannot allocate: the partials go to the
+    library's own fixed device array (ATTN_DECODE_NOALLOC_SCRATCH_BYTES), shared
+    by every call, so calls must not overlap on the GPU."""
+    B, T, Hq, d = q.shape
+    max_blocks, num_blocks, cap, Hkv = _cache_geometry(k_cache, page_table)
+    if tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(o.shape) != (B, T, Hq, d):
+        raise ValueError("shape mismatch")
+    if lse is not None and tuple(lse.shape) != (B, Hq, T):
+        raise ValueError("lse must be [B, Hq, T]")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    st = lib.attn_decode_noalloc(_dev(q, "q", torch.bfloat16), _dev(k_cache, "k_cache", torch.bfloat16),
+                                 _dev(v_cache, "v_cache", torch.bfloat16), _dev(seqlens_k, "seqlens_k", torch.int32),
+                                 None if page_table is None else _dev(page_table, "page_table", torch.int32),
+                                 max_blocks, num_blocks, cap, int(max_seqlen_k), _dev(o, "o"), _out_dtype(o),
+                                 None if lse is None else _dev(lse, "lse", torch.float32), B, T, Hq, Hkv, d, scale,
+                                 int(bool(causal)), int(num_splits), _stream(stream))
+    _check("attn_decode_noalloc", st)
 
 
 def kv_append(k_cache, v_cache, k_new, v_new, cache_lens, page_table=None, stream=None) -> None:
