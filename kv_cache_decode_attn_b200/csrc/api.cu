@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 #include <math.h>
 #include <stdio.h>
+#include <stdlib.h>
 
 #include <mutex>
 
@@ -96,7 +97,13 @@ bool decode_layout(int B, int T, int Hq, int Hkv, int d, int max_seqlen_k, int n
   return true;
 }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA; }
+// With KVATTN_DEBUG set in the environment, CUDA failures are also printed to stderr.
+int cuda_status(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return ATTN_OK;
+  static const bool debug = getenv("KVATTN_DEBUG") != nullptr;
+  if (debug) fprintf(stderr, "[kvattn] %s: %s (%d)\n", where, cudaGetErrorString(e), (int)e);
+  return ATTN_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -170,7 +177,7 @@ int attn_prefill(const void* q, const void* k, const void* v, void* o, int o_dty
   a.scale = scale;
   a.causal = causal;
   a.status = st;
-  return cuda_status(launch_prefill(a, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_prefill(a, static_cast<cudaStream_t>(stream)), "attn_prefill");
 }
 
 int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens_k,
@@ -227,7 +234,7 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
   a.part_o = static_cast<float*>(workspace);
   a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + L.lse_offset);
   a.status = st;
-  return cuda_status(launch_decode(a, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_decode(a, static_cast<cudaStream_t>(stream)), "attn_decode");
 }
 
 int kv_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new, const int32_t* cache_lens,
@@ -260,7 +267,7 @@ int kv_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new
   a.Hkv = Hkv;
   a.d = d;
   a.status = st;
-  return cuda_status(launch_append(a, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_append(a, static_cast<cudaStream_t>(stream)), "kv_append");
 }
 
 }  // extern "C"

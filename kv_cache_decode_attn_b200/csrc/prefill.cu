@@ -1,14 +1,20 @@
 // Prefill attention on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
 //
-// One CTA computes a 128-row query tile of one (batch, query head).  Warp roles:
-//   warps 0-3  softmax / correction / epilogue: thread i owns query row i, which
-//              is TMEM lane i of the S and O accumulators;
-//   warp 4     TMA producer: Q once, then K_j and V_j tiles into a 2-stage ring;
-//   warp 5     MMA issuer: S_j = Q K_j^T into one of two TMEM S buffers, and
-//              O += P_j V_j into the TMEM O accumulator.
-// S is double-buffered, so the tensor core computes S_{j+1} while the softmax
-// warps turn S_j into P_j.  P_j (bf16) goes to shared memory in the K-major
-// 128-byte-swizzled layout the MMA reads as its A operand.
+// One CTA computes two 128-row query tiles (A: rows 256*qb .. +127, B: the next
+// 128) of one (batch, query head); both tiles share every K/V tile it loads.
+// Warp roles:
+//   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread i of a
+//              group owns query row i, which is TMEM lane i of its S and O;
+//   warp 8     TMA producer: Q_A and Q_B once, then K_j, V_j into a 2-stage ring;
+//   warp 9     MMA issuer (one thread).
+// TMEM (512 columns): S_A | S_B | O_A | O_B.  Each softmax group reads its S row,
+// turns it into bf16 probabilities P and writes P back over the first half of
+// the same S columns; the PV MMA reads P straight from TMEM as its A operand
+// (no shared-memory round trip).  The MMA issue order
+//     PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), PV_A(j+1), ...
+// gives each softmax group the time of two MMAs to produce its next P.
+// Because MMAs complete in issue order, "S_X(j) complete" also means
+// "PV_X(j-1) complete", so a softmax group may rescale O_X as soon as it sees S_X(j).
 //
 // Online softmax (running maximum m and denominator l per row, base-2 exponent
 // with the scale folded in): a row's reference maximum is only raised when the
@@ -20,7 +26,8 @@
 // K/V tiles kept on chip; running softmax aggregation; write O once) and
 // "Numerical trick"; "大模型面試笔记——Attention篇" section 2 (online safe
 // softmax with the compensation factor); "[BEE-30062]" "背景" (FA2: scaling
-// moved out of the inner loop, parallel over query tiles).
+// moved out of the inner loop, parallel over query tiles; FA3: warp
+// specialisation with asynchronous TMA).
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -30,8 +37,9 @@
 namespace kvattn {
 namespace {
 
-constexpr int kBM = 128;          // query rows per CTA
-constexpr int kBN = 128;          // keys per tile
+constexpr int kBM = 128;          // query rows per tile (two tiles per CTA)
+constexpr int kBN = 128;          // keys per K/V tile
+constexpr int kThreads = 320;     // 8 softmax warps + TMA warp + MMA warp
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 of the largest allowed p
@@ -39,19 +47,19 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 of the largest allowed p
 template <int D>
 struct PrefillCfg {
   static constexpr int kHalves = D / 64;
-  static constexpr int kTileBytes = kBN * D * 2;          // one K or V tile (= one Q tile)
+  static constexpr int kTileBytes = kBN * D * 2;          // one Q, K or V tile
   static constexpr int kHalfBytes = kBN * 128;            // 128 rows x 128 B
-  static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + kTileBytes;
-  static constexpr int kVOff = kKOff + 2 * kTileBytes;
-  static constexpr int kPOff = kVOff + 2 * kTileBytes;
-  static constexpr int kPBytes = kBM * kBN * 2;
-  static constexpr int kBarOff = kPOff + kPBytes;
+  static constexpr int kQOff = 0;                         // Q_A, Q_B
+  static constexpr int kKOff = kQOff + 2 * kTileBytes;    // K stages 0, 1
+  static constexpr int kVOff = kKOff + 2 * kTileBytes;    // V stages 0, 1
+  static constexpr int kBarOff = kVOff + 2 * kTileBytes;
   static constexpr int kUsed = kBarOff + 256;
   // one CTA per SM: it owns all 512 TMEM columns
   static constexpr int kSmemBytes = (kUsed + 1024) > 120 * 1024 ? (kUsed + 1024) : 120 * 1024;
   static constexpr int kTmemCols = 512;
-  static constexpr int kSCol0 = 0, kSCol1 = 128, kOCol = 256;
+  // TMEM columns: S of tile t at 128*t, O of tile t at 256 + D*t
+  __host__ __device__ static constexpr int s_col(int t) { return 128 * t; }
+  __host__ __device__ static constexpr int o_col(int t) { return 256 + D * t; }
 };
 
 enum Bar {
@@ -59,10 +67,9 @@ enum Bar {
   B_KFULL = 1,    // +stage
   B_VFULL = 3,    // +stage
   B_KVEMPTY = 5,  // +stage
-  B_SFULL = 7,    // +buffer
-  B_SFREE = 9,    // +buffer
-  B_PFULL = 11,
-  B_ODONE = 12,
+  B_SFULL = 7,    // +tile
+  B_PFULL = 9,    // +tile
+  B_ODONE = 11,   // +tile
   B_DRAIN = 13,   // only used when a bounded wait gave up
   B_COUNT = 14
 };
@@ -71,7 +78,7 @@ struct PrefillParams {
   void* o;
   float* lse;
   unsigned* status;
-  int N, Hq, Hkv, G, n_qtiles;
+  int N, Hq, Hkv, G, n_qblocks, n_ktiles;
   float scale_log2;
   int causal, o_bf16;
 };
@@ -86,7 +93,7 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
   using C = PrefillCfg<D>;
@@ -98,9 +105,11 @@ __global__ void __launch_bounds__(192, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.x, b = blockIdx.y;
-  const int qt = p.n_qtiles - 1 - blockIdx.z;      // heaviest causal tiles launch first
+  const int qb = p.n_qblocks - 1 - blockIdx.z;      // heaviest causal blocks launch first
   const int kvh = h / p.G;
-  const int n_kv = p.causal ? (qt + 1) : (p.N + kBN - 1) / kBN;
+  // K/V tiles each query tile needs
+  const int n_kv0 = p.causal ? min(2 * qb + 1, p.n_ktiles) : p.n_ktiles;
+  const int n_load = p.causal ? min(2 * qb + 2, p.n_ktiles) : p.n_ktiles;   // = tile B's count, >= n_kv0
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[B_Q], 1);
@@ -109,10 +118,9 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&bars[B_VFULL + s], 1);
       mbar_init(&bars[B_KVEMPTY + s], 1);
       mbar_init(&bars[B_SFULL + s], 1);
-      mbar_init(&bars[B_SFREE + s], 4);
+      mbar_init(&bars[B_PFULL + s], 4);
+      mbar_init(&bars[B_ODONE + s], 1);
     }
-    mbar_init(&bars[B_PFULL], 4);
-    mbar_init(&bars[B_ODONE], 1);
     mbar_init(&bars[B_DRAIN], 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -126,20 +134,23 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------- TMA producer
     if (lane == 0) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      const uint64_t keep = policy_evict_last();    // K/V tiles are re-read by other query tiles
-      mbar_arrive_expect_tx(&bars[B_Q], C::kTileBytes);
+      const uint64_t keep = policy_evict_last();    // K/V tiles are re-read by other query blocks and heads
+      const uint64_t once = policy_evict_first();
+      mbar_arrive_expect_tx(&bars[B_Q], 2 * C::kTileBytes);
 #pragma unroll
-      for (int hh = 0; hh < C::kHalves; ++hh)
-        tma_load_4d(smem + C::kQOff + hh * C::kHalfBytes, &tmQ, &bars[B_Q], hh * 64, h, qt * kBM, b,
-                    policy_evict_first());
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int hh = 0; hh < C::kHalves; ++hh)
+          tma_load_4d(smem + C::kQOff + t * C::kTileBytes + hh * C::kHalfBytes, &tmQ, &bars[B_Q], hh * 64, h,
+                      (2 * qb + t) * kBM, b, once);
       int last_t[2] = {-1, -1};
-      for (int t = 0; t < n_kv; ++t) {
+      for (int t = 0; t < n_load; ++t) {
         const int st = t & 1;
         if (t >= 2 && !wait_or_abort(&bars[B_KVEMPTY + st], ((t >> 1) - 1) & 1, abort_flag, p.status)) break;
         last_t[st] = t;
@@ -162,88 +173,98 @@ __global__ void __launch_bounds__(192, 1)
         mbar_wait(&bars[B_VFULL + st], (last_t[st] >> 1) & 1);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(kBM, kBN, 0, 0);     // Q (K-major) x K^T (K-major)
-      constexpr uint32_t idO = idesc_bf16(kBM, D, 0, 1);       // P (K-major) x V (N-major)
-      const uint32_t q_s = smem_u32(smem + C::kQOff);
-      const uint32_t p_s = smem_u32(smem + C::kPOff);
-      auto issue_s = [&](int t) {
-        const int st = t & 1;
-        const uint32_t k_s = smem_u32(smem + C::kKOff + st * C::kTileBytes);
-        const uint32_t d_tmem = tmem + (st ? C::kSCol1 : C::kSCol0);
+      constexpr uint32_t idO = idesc_bf16(kBM, D, 0, 1);       // P (TMEM) x V (N-major)
+      auto issue_s = [&](int t, int j) {      // S_t = Q_t K_j^T
+        const uint32_t q_s = smem_u32(smem + C::kQOff + t * C::kTileBytes);
+        const uint32_t k_s = smem_u32(smem + C::kKOff + (j & 1) * C::kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
-          tc_mma_ss(d_tmem, smem_desc(q_s + off, 16, 1024), smem_desc(k_s + off, 16, 1024), idS, kk > 0);
+          tc_mma_ss(tmem + C::s_col(t), smem_desc(q_s + off, 16, 1024), smem_desc(k_s + off, 16, 1024), idS, kk > 0);
         }
-        tc_commit(&bars[B_SFULL + st]);
+        tc_commit(&bars[B_SFULL + t]);
+      };
+      auto issue_pv = [&](int t, int j) {     // O_t += P_t V_j, P_t in the first 64 columns of S_t
+        const uint32_t v_s = smem_u32(smem + C::kVOff + (j & 1) * C::kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          tc_mma_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8, smem_desc(v_s + kk * 16 * 128, C::kHalfBytes, 1024),
+                    idO, (j > 0 || kk > 0) ? 1u : 0u);
       };
       bool ok = wait_or_abort(&bars[B_Q], 0, abort_flag, p.status) &&
                 wait_or_abort(&bars[B_KFULL], 0, abort_flag, p.status);
       if (ok) {
         tc_fence_after();
-        issue_s(0);
+        issue_s(0, 0);
+        issue_s(1, 0);
       }
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int t = j + 1;
-        if (t < n_kv) {
-          ok = wait_or_abort(&bars[B_KFULL + (t & 1)], (t >> 1) & 1, abort_flag, p.status) &&
-               (t < 2 || wait_or_abort(&bars[B_SFREE + (t & 1)], ((t >> 1) - 1) & 1, abort_flag, p.status));
+      for (int j = 0; ok && j < n_load; ++j) {
+        const int st = j & 1;
+        const bool next_k = j + 1 < n_load;
+        ok = wait_or_abort(&bars[B_VFULL + st], (j >> 1) & 1, abort_flag, p.status);
+        if (!ok) break;
+        if (j < n_kv0) {
+          ok = wait_or_abort(&bars[B_PFULL + 0], j & 1, abort_flag, p.status);
           if (!ok) break;
           tc_fence_after();
-          issue_s(t);
+          issue_pv(0, j);
+          if (j == n_kv0 - 1) tc_commit(&bars[B_ODONE + 0]);
         }
-        ok = wait_or_abort(&bars[B_PFULL], j & 1, abort_flag, p.status) &&
-             wait_or_abort(&bars[B_VFULL + (j & 1)], (j >> 1) & 1, abort_flag, p.status);
+        if (next_k) {
+          ok = wait_or_abort(&bars[B_KFULL + ((j + 1) & 1)], ((j + 1) >> 1) & 1, abort_flag, p.status);
+          if (!ok) break;
+          tc_fence_after();
+          if (j + 1 < n_kv0) issue_s(0, j + 1);
+        }
+        ok = wait_or_abort(&bars[B_PFULL + 1], j & 1, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t v_s = smem_u32(smem + C::kVOff + (j & 1) * C::kTileBytes);
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint32_t a_off = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
-          tc_mma_ss(tmem + C::kOCol, smem_desc(p_s + a_off, 16, 1024),
-                    smem_desc(v_s + kk * 16 * 128, C::kHalfBytes, 1024), idO, (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(&bars[B_ODONE]);
-        tc_commit(&bars[B_KVEMPTY + (j & 1)]);
+        issue_pv(1, j);
+        tc_commit(&bars[B_KVEMPTY + st]);       // K_j and V_j are no longer needed
+        if (j == n_load - 1) tc_commit(&bars[B_ODONE + 1]);
+        if (next_k) issue_s(1, j + 1);
       }
     }
   } else {
-    // ------------------------------------------------------ softmax warps 0-3
-    const int row = warp * 32 + lane;                   // TMEM lane == query row in the tile
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    const int q_row = qt * kBM + row;
+    // -------------------------------------------------- softmax warps 0-7
+    const int t = warp >> 2;                            // query tile of this group
+    const int row = (warp & 3) * 32 + lane;             // TMEM lane == query row in the tile
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t s_addr = lane_base + C::s_col(t);
+    const uint32_t o_addr = lane_base + C::o_col(t);
+    const int q_row = (2 * qb + t) * kBM + row;
+    const int nkv = t ? n_load : n_kv0;
     float m = -INFINITY, l = 0.f;
-    uint8_t* p_tile = smem + C::kPOff;
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      const int sb = j & 1;
-      if (!wait_or_abort(&bars[B_SFULL + sb], (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+    for (int j = 0; j < nkv; ++j) {
+      if (!wait_or_abort(&bars[B_SFULL + t], j & 1, abort_flag, p.status)) { ok = false; break; }
       tc_fence_after();
       float s[kBN];
 #pragma unroll
       for (int c = 0; c < kBN; c += 32) {
         uint32_t r[32];
-        tmem_ld32(lane_base + (sb ? C::kSCol1 : C::kSCol0) + c, r);
+        tmem_ld32(s_addr + c, r);
 #pragma unroll
         for (int e = 0; e < 32; ++e) s[c + e] = __uint_as_float(r[e]);
       }
       tc_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[B_SFREE + sb]);
 
-      // mask: causal diagonal tile, or keys past N
+      // mask (causal diagonal tile, or keys past N) and the row maximum of the raw scores
       const int key0 = j * kBN;
       const int lim = p.causal ? min(q_row - key0 + 1, p.N - key0) : (p.N - key0);   // visible keys: [0, lim)
-      float mx = -INFINITY;
+      if (lim < kBN) {
 #pragma unroll
-      for (int c = 0; c < kBN; ++c) {
-        s[c] = (c < lim) ? s[c] * p.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < kBN; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
       }
+      float mx = max3f(s[0], s[1], s[2]);
+#pragma unroll
+      for (int c = 3; c + 1 < kBN; c += 2) mx = max3f(mx, s[c], s[c + 1]);
+      mx = fmaxf(mx, s[kBN - 1]);
+      mx *= p.scale_log2;                                      // scores in log2 units
       const bool raise = mx > m + kRescaleThreshold;          // also true on the first tile (m = -inf)
       const bool warp_raise = __any_sync(0xffffffffu, raise);
       float alpha = 1.f;
@@ -252,49 +273,42 @@ __global__ void __launch_bounds__(192, 1)
         alpha = ex2(m - m_new);                                 // 0 when m == -inf
         m = m_new;
       }
-      const float mu = (m == -INFINITY) ? 0.f : m;
+      const float neg_mu = (m == -INFINITY) ? 0.f : -m;
       float ls = 0.f;
-      uint32_t pk[kBN / 2];
 #pragma unroll
-      for (int c = 0; c < kBN; c += 2) {
-        const float p0 = ex2(s[c] - mu), p1 = ex2(s[c + 1] - mu);
-        ls += p0 + p1;
-        pk[c / 2] = pack_bf16x2(p0, p1);
+      for (int c = 0; c < kBN; c += 16) {
+        uint32_t pk[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          const float p0 = ex2(fmaf(s[c + e], p.scale_log2, neg_mu));
+          const float p1 = ex2(fmaf(s[c + e + 1], p.scale_log2, neg_mu));
+          ls += p0 + p1;
+          pk[e / 2] = pack_bf16x2(p0, p1);
+        }
+        tmem_st8(s_addr + c / 2, pk);           // P row over the consumed S columns
       }
       l = l * alpha + ls;
-
-      // PV of the previous tile must be done before P and O are touched
-      if (j > 0) {
-        if (!wait_or_abort(&bars[B_ODONE], (j - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-        tc_fence_after();
-        if (warp_raise) {
+      // O_t is stable here (PV_t(j-1) completed before S_t(j) did) and PV_t(j)
+      // waits for this group's arrival below
+      if (warp_raise && j > 0) {
 #pragma unroll
-          for (int c = 0; c < D; c += 32) {
-            uint32_t r[32];
-            tmem_ld32(lane_base + C::kOCol + c, r);
-            tc_wait_ld();
+        for (int c = 0; c < D; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(o_addr + c, r);
+          tc_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            tmem_st32(lane_base + C::kOCol + c, r);
-          }
-          tc_wait_st();
+          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tmem_st32(o_addr + c, r);
         }
       }
-      // P row -> shared memory, K-major with the 128-byte swizzle (two 64-key halves)
-#pragma unroll
-      for (int ch = 0; ch < kBN / 8; ++ch) {
-        const int half = ch >> 3, cw = ch & 7;
-        uint4 v = make_uint4(pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
-        *reinterpret_cast<uint4*>(p_tile + half * (kBM * 128) + row * 128 + ((cw ^ (row & 7)) << 4)) = v;
-      }
-      fence_proxy_async_smem();
+      tc_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[B_PFULL]);
+      if (lane == 0) mbar_arrive(&bars[B_PFULL + t]);
     }
 
     // ---------------------------------------------------------- epilogue
-    if (ok && wait_or_abort(&bars[B_ODONE], (n_kv - 1) & 1, abort_flag, p.status)) {
+    if (ok && wait_or_abort(&bars[B_ODONE + t], 0, abort_flag, p.status)) {
       tc_fence_after();
       const float inv_l = 1.f / l;
       const bool store = q_row < p.N;
@@ -302,7 +316,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         uint32_t r[32];
-        tmem_ld32(lane_base + C::kOCol + c, r);
+        tmem_ld32(o_addr + c, r);
         tc_wait_ld();
         if (store) {
           if (p.o_bf16) {
@@ -331,7 +345,7 @@ __global__ void __launch_bounds__(192, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (*abort_flag && warp == 5 && lane == 0) {
+  if (*abort_flag && warp == 9 && lane == 0) {
     // a wait gave up: let every tensor-core op this CTA issued drain before TMEM is released
     tc_commit(&bars[B_DRAIN]);
     mbar_wait(&bars[B_DRAIN], 0);
@@ -363,15 +377,16 @@ cudaError_t run_prefill(const PrefillLaunch& a, cudaStream_t stream) {
   p.Hq = a.Hq;
   p.Hkv = a.Hkv;
   p.G = a.Hq / a.Hkv;
-  p.n_qtiles = (a.N + kBM - 1) / kBM;
+  p.n_qblocks = (a.N + 2 * kBM - 1) / (2 * kBM);
+  p.n_ktiles = (a.N + kBN - 1) / kBN;
   p.scale_log2 = a.scale * kLog2e;
   p.causal = a.causal;
   p.o_bf16 = a.o_bf16;
   auto kern = prefill_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.Hq, a.B, p.n_qtiles);
-  kern<<<grid, 192, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  dim3 grid(a.Hq, a.B, p.n_qblocks);
+  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
