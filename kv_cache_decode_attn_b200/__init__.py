@@ -5,7 +5,7 @@ Python binding of ``libkvattn.so``: the functions below carry the C-ABI names of
 current CUDA stream) from torch tensors.  Every step of the computation runs in
 the library's CUDA kernels; there is no CPU or library fallback, and importing
 this package fails if the library has not been built
-(``python -m kv_cache_decode_attn_b200.build``).
+(``python kv_cache_decode_attn_b200/build.py``).
 
 The raw ctypes handle is ``lib``; tests call through it or through these wrappers.
 """
@@ -53,7 +53,7 @@ _SIGNATURES = {
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m kv_cache_decode_attn_b200.build`")
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python kv_cache_decode_attn_b200/build.py`")
     handle = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in _SIGNATURES.items():
         fn = getattr(handle, name)

@@ -1,6 +1,6 @@
 """Build ``libkvattn.so`` in-tree with nvcc for sm_100a.
 
-``python -m kv_cache_decode_attn_b200.build`` (or ``build()``) compiles every
+``python kv_cache_decode_attn_b200/build.py`` (or ``build()``) compiles every
 ``csrc/*.cu`` file into one shared library beside this file.  The library links
 the CUDA runtime statically and reaches the driver API (tensor-map encoding)
 through ``cudaGetDriverEntryPointByVersion``, so it needs no ``-lcuda`` at link

@@ -260,10 +260,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < kBN; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
       }
-      float mx = max3f(s[0], s[1], s[2]);
+      float mx8[8];
 #pragma unroll
-      for (int c = 3; c + 1 < kBN; c += 2) mx = max3f(mx, s[c], s[c + 1]);
-      mx = fmaxf(mx, s[kBN - 1]);
+      for (int i = 0; i < 8; ++i) mx8[i] = max3f(s[i], s[i + 8], s[i + 16]);
+#pragma unroll
+      for (int c = 24; c + 8 < kBN; c += 16)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx8[i] = max3f(mx8[i], s[c + i], s[c + 8 + i]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(mx8[i], s[kBN - 8 + i]);
+      float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
       mx *= p.scale_log2;                                      // scores in log2 units
       const bool raise = mx > m + kRescaleThreshold;          // also true on the first tile (m = -inf)
       const bool warp_raise = __any_sync(0xffffffffu, raise);
@@ -274,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         m = m_new;
       }
       const float neg_mu = (m == -INFINITY) ? 0.f : -m;
-      float ls = 0.f;
+      float ls4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < kBN; c += 16) {
         uint32_t pk[8];
@@ -282,11 +288,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 16; e += 2) {
           const float p0 = ex2(fmaf(s[c + e], p.scale_log2, neg_mu));
           const float p1 = ex2(fmaf(s[c + e + 1], p.scale_log2, neg_mu));
-          ls += p0 + p1;
+          ls4[(e >> 1) & 3] += p0 + p1;
           pk[e / 2] = pack_bf16x2(p0, p1);
         }
         tmem_st8(s_addr + c / 2, pk);           // P row over the consumed S columns
       }
+      const float ls = (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
       l = l * alpha + ls;
       // O_t is stable here (PV_t(j-1) completed before S_t(j) did) and PV_t(j)
       // waits for this group's arrival below
