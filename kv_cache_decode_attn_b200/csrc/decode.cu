@@ -366,9 +366,30 @@ __global__ void __launch_bounds__(DecodeCfg<D, MT>::kThreads, DecodeCfg<D, MT>::
   }
 }
 
+// kPer consecutive partial-output floats of one lane (2 or 4), as a float4.
+template <int kPer>
+__device__ __forceinline__ float4 load_part(const float* src) {
+  if constexpr (kPer == 4) {
+    return __ldg(reinterpret_cast<const float4*>(src));
+  } else {
+    const float2 v = __ldg(reinterpret_cast<const float2*>(src));
+    return make_float4(v.x, v.y, 0.f, 0.f);
+  }
+}
+
+template <int kPer>
+__device__ __forceinline__ void accumulate(float (&acc)[kPer], float w, float4 x) {
+  acc[0] = fmaf(w, x.x, acc[0]);
+  acc[1] = fmaf(w, x.y, acc[1]);
+  if constexpr (kPer == 4) {
+    acc[2] = fmaf(w, x.z, acc[2]);
+    acc[3] = fmaf(w, x.w, acc[3]);
+  }
+}
+
 // One warp per output row (b, t, h): merge the chunk partials of that row.
 template <int D>
-__global__ void __launch_bounds__(256) decode_combine_kernel(const float* __restrict__ part_o,
+__global__ void __launch_bounds__(256, 4) decode_combine_kernel(const float* __restrict__ part_o,
                                                              const float* __restrict__ part_lse,
                                                              const int32_t* __restrict__ seqlens, void* o, int o_bf16,
                                                              float* lse, SplitParams p, int B, int paged) {
@@ -406,20 +427,30 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const float* __rest
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
     lse_row = M + logf(z);
-    for (int c = 0; c < nc; ++c) {
-      const float lc = part_lse[(item0 + c) * p.R + r];
-      if (lc == -INFINITY) continue;
-      const float w = expf(lc - lse_row);
-      const float* src = part_o + ((item0 + c) * p.R + r) * D + lane * kPer;
-      if constexpr (kPer == 4) {
-        const float4 x = *reinterpret_cast<const float4*>(src);
-        acc[0] += w * x.x;
-        acc[1] += w * x.y;
-        acc[2] += w * x.z;
-        acc[3] += w * x.w;
-      } else {
+    // lanes compute the weights of 32 chunks at a time; every lane then walks
+    // those chunks with several independent loads in flight
+    const float* src0 = part_o + (item0 * p.R + r) * D + lane * kPer;
+    const size_t cstride = (size_t)p.R * D;     // floats between consecutive chunks of this row
+    for (int c0 = 0; c0 < nc; c0 += 32) {
+      const int c = c0 + lane;
+      const float lc = c < nc ? part_lse[(item0 + c) * p.R + r] : -INFINITY;
+      const float wl = (lc == -INFINITY) ? 0.f : expf(lc - lse_row);
+      const int n = min(32, nc - c0);
+      int i = 0;
+      for (; i + 4 <= n; i += 4) {
+        float w[4];
+        float4 x[4];
 #pragma unroll
-        for (int e = 0; e < kPer; ++e) acc[e] += w * src[e];
+        for (int u = 0; u < 4; ++u) {
+          w[u] = __shfl_sync(0xffffffffu, wl, i + u);
+          x[u] = load_part<kPer>(src0 + (size_t)(c0 + i + u) * cstride);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) accumulate<kPer>(acc, w[u], x[u]);
+      }
+      for (; i < n; ++i) {
+        const float w = __shfl_sync(0xffffffffu, wl, i);
+        accumulate<kPer>(acc, w, load_part<kPer>(src0 + (size_t)(c0 + i) * cstride));
       }
     }
   }
