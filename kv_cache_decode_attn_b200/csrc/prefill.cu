@@ -1,20 +1,25 @@
 // Prefill attention on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
 //
-// One CTA computes two 128-row query tiles (A: rows 256*qb .. +127, B: the next
-// 128) of one (batch, query head); both tiles share every K/V tile it loads.
-// Warp roles:
+// Persistent: one CTA per SM walks a list of work items, heaviest causal query
+// blocks first.  A work item is two 128-row query tiles (A: rows 256*qb .. +127,
+// B: the next 128) of one (batch, query head); both tiles share every K/V tile
+// loaded for the item.  Warp roles:
 //   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread i of a
 //              group owns query row i, which is TMEM lane i of its S and O;
-//   warp 8     TMA producer: Q_A and Q_B once, then K_j, V_j into a 2-stage ring;
+//   warp 8     TMA producer: Q_A and Q_B per item (the next item's Q is
+//              prefetched into L2 early), K_j and V_j through a 2-stage ring
+//              that runs on across items;
 //   warp 9     MMA issuer (one thread).
 // TMEM (512 columns): S_A | S_B | O_A | O_B.  Each softmax group reads its S row,
 // turns it into bf16 probabilities P and writes P back over the first half of
-// the same S columns; the PV MMA reads P straight from TMEM as its A operand
-// (no shared-memory round trip).  The MMA issue order
-//     PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), PV_A(j+1), ...
-// gives each softmax group the time of two MMAs to produce its next P.
-// Because MMAs complete in issue order, "S_X(j) complete" also means
-// "PV_X(j-1) complete", so a softmax group may rescale O_X as soon as it sees S_X(j).
+// the same S columns; the PV MMA reads P straight from TMEM as its A operand.
+// The MMA issue order  PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), PV_A(j+1), ...
+// gives each softmax group the time of two MMAs to produce its next P.  Because
+// MMAs complete in issue order, "S_X(j) complete" also means "PV_X(j-1)
+// complete", so a softmax group may rescale O_X as soon as it sees S_X(j).  At
+// an item boundary the next item's first S MMAs run while the softmax warps
+// write out the previous item's O; the first PV of the new item waits until
+// that O has been read (O_FREE).
 //
 // Online softmax (running maximum m and denominator l per row, base-2 exponent
 // with the scale folded in): a row's reference maximum is only raised when the
@@ -63,22 +68,24 @@ struct PrefillCfg {
 };
 
 enum Bar {
-  B_Q = 0,
-  B_KFULL = 1,    // +stage
-  B_VFULL = 3,    // +stage
-  B_KVEMPTY = 5,  // +stage
-  B_SFULL = 7,    // +tile
-  B_PFULL = 9,    // +tile
-  B_ODONE = 11,   // +tile
-  B_DRAIN = 13,   // only used when a bounded wait gave up
-  B_COUNT = 14
+  B_QFULL = 0,
+  B_QEMPTY = 1,   // all MMAs of an item done: its Q tiles may be replaced
+  B_KFULL = 2,    // +stage
+  B_VFULL = 4,    // +stage
+  B_KVEMPTY = 6,  // +stage
+  B_SFULL = 8,    // +tile
+  B_PFULL = 10,   // +tile
+  B_ODONE = 12,   // +tile: last PV of an item done
+  B_OFREE = 14,   // +tile: the softmax group has read O out
+  B_DRAIN = 16,   // only used when a bounded wait gave up
+  B_COUNT = 17
 };
 
 struct PrefillParams {
   void* o;
   float* lse;
   unsigned* status;
-  int N, Hq, Hkv, G, n_qblocks, n_ktiles;
+  int B, N, Hq, Hkv, G, n_qblocks, n_ktiles, n_items;
   float scale_log2;
   int causal, o_bf16;
 };
@@ -90,6 +97,24 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
   atomicOr(status, DEV_TIMEOUT);
   *abort_flag = 1;
   return false;
+}
+
+struct Item {
+  int qb, h, b, n_kv0, n_load;   // n_kv0: K/V tiles of query tile A; n_load: of tile B (>= n_kv0)
+};
+
+// Work item w: heaviest causal query blocks first, then consecutive heads (the
+// query heads of one K/V head are adjacent, so its K/V tiles are reused from L2).
+__device__ __forceinline__ Item item_of(int w, const PrefillParams& p) {
+  Item it;
+  const int per = p.Hq * p.B;
+  it.qb = p.n_qblocks - 1 - w / per;
+  const int r = w - (w / per) * per;
+  it.h = r % p.Hq;
+  it.b = r / p.Hq;
+  it.n_kv0 = p.causal ? min(2 * it.qb + 1, p.n_ktiles) : p.n_ktiles;
+  it.n_load = p.causal ? min(2 * it.qb + 2, p.n_ktiles) : p.n_ktiles;
+  return it;
 }
 
 template <int D>
@@ -104,15 +129,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int qb = p.n_qblocks - 1 - blockIdx.z;      // heaviest causal blocks launch first
-  const int kvh = h / p.G;
-  // K/V tiles each query tile needs
-  const int n_kv0 = p.causal ? min(2 * qb + 1, p.n_ktiles) : p.n_ktiles;
-  const int n_load = p.causal ? min(2 * qb + 2, p.n_ktiles) : p.n_ktiles;   // = tile B's count, >= n_kv0
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars[B_Q], 1);
+    mbar_init(&bars[B_QFULL], 1);
+    mbar_init(&bars[B_QEMPTY], 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[B_KFULL + s], 1);
       mbar_init(&bars[B_VFULL + s], 1);
@@ -120,6 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars[B_SFULL + s], 1);
       mbar_init(&bars[B_PFULL + s], 4);
       mbar_init(&bars[B_ODONE + s], 1);
+      mbar_init(&bars[B_OFREE + s], 4);
     }
     mbar_init(&bars[B_DRAIN], 1);
     *abort_flag = 0;
@@ -142,35 +163,53 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmV);
       const uint64_t keep = policy_evict_last();    // K/V tiles are re-read by other query blocks and heads
       const uint64_t once = policy_evict_first();
-      mbar_arrive_expect_tx(&bars[B_Q], 2 * C::kTileBytes);
+      int g = 0, it = 0, q_loaded = 0;              // K/V tiles loaded, items started, Q loads issued
+      int last_g[2] = {-1, -1};
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x, ++it) {
+        const Item itm = item_of(w, p);
+        const int kvh = itm.h / p.G;
+        if (it > 0 && !wait_or_abort(&bars[B_QEMPTY], (it - 1) & 1, abort_flag, p.status)) break;
+        mbar_arrive_expect_tx(&bars[B_QFULL], 2 * C::kTileBytes);
+        ++q_loaded;
 #pragma unroll
-      for (int t = 0; t < 2; ++t)
+        for (int t = 0; t < 2; ++t)
 #pragma unroll
-        for (int hh = 0; hh < C::kHalves; ++hh)
-          tma_load_4d(smem + C::kQOff + t * C::kTileBytes + hh * C::kHalfBytes, &tmQ, &bars[B_Q], hh * 64, h,
-                      (2 * qb + t) * kBM, b, once);
-      int last_t[2] = {-1, -1};
-      for (int t = 0; t < n_load; ++t) {
-        const int st = t & 1;
-        if (t >= 2 && !wait_or_abort(&bars[B_KVEMPTY + st], ((t >> 1) - 1) & 1, abort_flag, p.status)) break;
-        last_t[st] = t;
-        mbar_arrive_expect_tx(&bars[B_KFULL + st], C::kTileBytes);
+          for (int hh = 0; hh < C::kHalves; ++hh)
+            tma_load_4d(smem + C::kQOff + t * C::kTileBytes + hh * C::kHalfBytes, &tmQ, &bars[B_QFULL], hh * 64,
+                        itm.h, (2 * itm.qb + t) * kBM, itm.b, once);
+        if (w + (int)gridDim.x < p.n_items) {       // warm L2 with the next item's Q
+          const Item nx = item_of(w + gridDim.x, p);
 #pragma unroll
-        for (int hh = 0; hh < C::kHalves; ++hh)
-          tma_load_4d(smem + C::kKOff + st * C::kTileBytes + hh * C::kHalfBytes, &tmK, &bars[B_KFULL + st], hh * 64,
-                      kvh, t * kBN, b, keep);
-        mbar_arrive_expect_tx(&bars[B_VFULL + st], C::kTileBytes);
+          for (int t = 0; t < 2; ++t)
 #pragma unroll
-        for (int hh = 0; hh < C::kHalves; ++hh)
-          tma_load_4d(smem + C::kVOff + st * C::kTileBytes + hh * C::kHalfBytes, &tmV, &bars[B_VFULL + st], hh * 64,
-                      kvh, t * kBN, b, keep);
+            for (int hh = 0; hh < C::kHalves; ++hh) tma_prefetch_4d(&tmQ, hh * 64, nx.h, (2 * nx.qb + t) * kBM, nx.b);
+        }
+        for (int t = 0; t < itm.n_load; ++t, ++g) {
+          const int st = g & 1;
+          if (g >= 2 && !wait_or_abort(&bars[B_KVEMPTY + st], ((g >> 1) - 1) & 1, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          last_g[st] = g;
+          mbar_arrive_expect_tx(&bars[B_KFULL + st], C::kTileBytes);
+#pragma unroll
+          for (int hh = 0; hh < C::kHalves; ++hh)
+            tma_load_4d(smem + C::kKOff + st * C::kTileBytes + hh * C::kHalfBytes, &tmK, &bars[B_KFULL + st],
+                        hh * 64, kvh, t * kBN, itm.b, keep);
+          mbar_arrive_expect_tx(&bars[B_VFULL + st], C::kTileBytes);
+#pragma unroll
+          for (int hh = 0; hh < C::kHalves; ++hh)
+            tma_load_4d(smem + C::kVOff + st * C::kTileBytes + hh * C::kHalfBytes, &tmV, &bars[B_VFULL + st],
+                        hh * 64, kvh, t * kBN, itm.b, keep);
+        }
       }
       // no copy may still be landing in shared memory when the CTA exits
-      mbar_wait(&bars[B_Q], 0);
+      if (q_loaded > 0) mbar_wait(&bars[B_QFULL], (q_loaded - 1) & 1);
       for (int st = 0; st < 2; ++st) {
-        if (last_t[st] < 0) continue;
-        mbar_wait(&bars[B_KFULL + st], (last_t[st] >> 1) & 1);
-        mbar_wait(&bars[B_VFULL + st], (last_t[st] >> 1) & 1);
+        if (last_g[st] < 0) continue;
+        mbar_wait(&bars[B_KFULL + st], (last_g[st] >> 1) & 1);
+        mbar_wait(&bars[B_VFULL + st], (last_g[st] >> 1) & 1);
       }
     }
   } else if (warp == 9) {
@@ -178,9 +217,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(kBM, kBN, 0, 0);     // Q (K-major) x K^T (K-major)
       constexpr uint32_t idO = idesc_bf16(kBM, D, 0, 1);       // P (TMEM) x V (N-major)
-      auto issue_s = [&](int t, int j) {      // S_t = Q_t K_j^T
+      auto issue_s = [&](int t, int st) {     // S_t = Q_t K^T, K in ring stage st
         const uint32_t q_s = smem_u32(smem + C::kQOff + t * C::kTileBytes);
-        const uint32_t k_s = smem_u32(smem + C::kKOff + (j & 1) * C::kTileBytes);
+        const uint32_t k_s = smem_u32(smem + C::kKOff + st * C::kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
@@ -188,45 +227,60 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_commit(&bars[B_SFULL + t]);
       };
-      auto issue_pv = [&](int t, int j) {     // O_t += P_t V_j, P_t in the first 64 columns of S_t
-        const uint32_t v_s = smem_u32(smem + C::kVOff + (j & 1) * C::kTileBytes);
+      auto issue_pv = [&](int t, int st, bool first) {   // O_t (+)= P_t V, P_t in the first 64 columns of S_t
+        const uint32_t v_s = smem_u32(smem + C::kVOff + st * C::kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
           tc_mma_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8, smem_desc(v_s + kk * 16 * 128, C::kHalfBytes, 1024),
-                    idO, (j > 0 || kk > 0) ? 1u : 0u);
+                    idO, (!first || kk > 0) ? 1u : 0u);
       };
-      bool ok = wait_or_abort(&bars[B_Q], 0, abort_flag, p.status) &&
-                wait_or_abort(&bars[B_KFULL], 0, abort_flag, p.status);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        issue_s(1, 0);
-      }
-      for (int j = 0; ok && j < n_load; ++j) {
-        const int st = j & 1;
-        const bool next_k = j + 1 < n_load;
-        ok = wait_or_abort(&bars[B_VFULL + st], (j >> 1) & 1, abort_flag, p.status);
-        if (!ok) break;
-        if (j < n_kv0) {
-          ok = wait_or_abort(&bars[B_PFULL + 0], j & 1, abort_flag, p.status);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv(0, j);
-          if (j == n_kv0 - 1) tc_commit(&bars[B_ODONE + 0]);
-        }
-        if (next_k) {
-          ok = wait_or_abort(&bars[B_KFULL + ((j + 1) & 1)], ((j + 1) >> 1) & 1, abort_flag, p.status);
-          if (!ok) break;
-          tc_fence_after();
-          if (j + 1 < n_kv0) issue_s(0, j + 1);
-        }
-        ok = wait_or_abort(&bars[B_PFULL + 1], j & 1, abort_flag, p.status);
+      int g = 0, it = 0;                     // K/V tiles consumed, items done
+      int pcnt[2] = {0, 0};                  // P_FULL phases consumed per tile
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x, ++it) {
+        const Item itm = item_of(w, p);
+        const int g0 = g;
+        ok = wait_or_abort(&bars[B_QFULL], it & 1, abort_flag, p.status) &&
+             wait_or_abort(&bars[B_KFULL + (g0 & 1)], (g0 >> 1) & 1, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
-        issue_pv(1, j);
-        tc_commit(&bars[B_KVEMPTY + st]);       // K_j and V_j are no longer needed
-        if (j == n_load - 1) tc_commit(&bars[B_ODONE + 1]);
-        if (next_k) issue_s(1, j + 1);
+        issue_s(0, g0 & 1);
+        issue_s(1, g0 & 1);
+        for (int j = 0; j < itm.n_load; ++j) {
+          const int gj = g0 + j, st = gj & 1;
+          const bool next_k = j + 1 < itm.n_load;
+          ok = wait_or_abort(&bars[B_VFULL + st], (gj >> 1) & 1, abort_flag, p.status);
+          if (!ok) break;
+          if (j < itm.n_kv0) {
+            ok = wait_or_abort(&bars[B_PFULL + 0], (pcnt[0]++) & 1, abort_flag, p.status) &&
+                 (j > 0 || it == 0 || wait_or_abort(&bars[B_OFREE + 0], (it - 1) & 1, abort_flag, p.status));
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(0, st, j == 0);
+            if (j == itm.n_kv0 - 1) tc_commit(&bars[B_ODONE + 0]);
+          }
+          if (next_k) {
+            ok = wait_or_abort(&bars[B_KFULL + ((gj + 1) & 1)], ((gj + 1) >> 1) & 1, abort_flag, p.status);
+            if (!ok) break;
+            tc_fence_after();
+            if (j + 1 < itm.n_kv0) issue_s(0, (gj + 1) & 1);
+          }
+          ok = wait_or_abort(&bars[B_PFULL + 1], (pcnt[1]++) & 1, abort_flag, p.status) &&
+               (j > 0 || it == 0 || wait_or_abort(&bars[B_OFREE + 1], (it - 1) & 1, abort_flag, p.status));
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(1, st, j == 0);
+          tc_commit(&bars[B_KVEMPTY + st]);       // K and V of this stage are no longer needed
+          if (j == itm.n_load - 1) tc_commit(&bars[B_ODONE + 1]);
+          if (next_k) {
+            issue_s(1, (gj + 1) & 1);
+            // that was the item's last MMA reading Q: the next item's Q may land once it is done
+            if (j + 2 == itm.n_load) tc_commit(&bars[B_QEMPTY]);
+          }
+        }
+        if (!ok) break;
+        if (itm.n_load == 1) tc_commit(&bars[B_QEMPTY]);
+        g = g0 + itm.n_load;
       }
     }
   } else {
@@ -236,12 +290,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t s_addr = lane_base + C::s_col(t);
     const uint32_t o_addr = lane_base + C::o_col(t);
-    const int q_row = (2 * qb + t) * kBM + row;
-    const int nkv = t ? n_load : n_kv0;
-    float m = -INFINITY, l = 0.f;
+    int scnt = 0, it = 0;                               // S_FULL phases consumed, items done
     bool ok = true;
+    for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x, ++it) {
+    const Item itm = item_of(w, p);
+    const int q_row = (2 * itm.qb + t) * kBM + row;
+    const int nkv = t ? itm.n_load : itm.n_kv0;
+    float m = -INFINITY, l = 0.f;
     for (int j = 0; j < nkv; ++j) {
-      if (!wait_or_abort(&bars[B_SFULL + t], j & 1, abort_flag, p.status)) { ok = false; break; }
+      if (!wait_or_abort(&bars[B_SFULL + t], (scnt++) & 1, abort_flag, p.status)) { ok = false; break; }
       tc_fence_after();
       float s[kBN];
 #pragma unroll
@@ -315,11 +372,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---------------------------------------------------------- epilogue
-    if (ok && wait_or_abort(&bars[B_ODONE + t], 0, abort_flag, p.status)) {
+    if (!ok || !wait_or_abort(&bars[B_ODONE + t], it & 1, abort_flag, p.status)) {
+      ok = false;
+      break;
+    }
+    {
       tc_fence_after();
       const float inv_l = 1.f / l;
       const bool store = q_row < p.N;
-      const size_t obase = (((size_t)b * p.N + q_row) * p.Hq + h) * D;
+      const size_t obase = (((size_t)itm.b * p.N + q_row) * p.Hq + itm.h) * D;
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         uint32_t r[32];
@@ -346,7 +407,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (store && p.lse) p.lse[((size_t)b * p.Hq + h) * p.N + q_row] = (m + log2f(l)) * kLn2;
+      if (store && p.lse) p.lse[((size_t)itm.b * p.Hq + itm.h) * p.N + q_row] = (m + log2f(l)) * kLn2;
+      // O_t has been read: the next item's first PV may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[B_OFREE + t]);
+    }
     }
   }
 
@@ -384,15 +450,23 @@ cudaError_t run_prefill(const PrefillLaunch& a, cudaStream_t stream) {
   p.Hq = a.Hq;
   p.Hkv = a.Hkv;
   p.G = a.Hq / a.Hkv;
+  p.B = a.B;
   p.n_qblocks = (a.N + 2 * kBM - 1) / (2 * kBM);
   p.n_ktiles = (a.N + kBN - 1) / kBN;
+  const long long items = (long long)p.n_qblocks * a.Hq * a.B;
+  if (items > INT32_MAX) return cudaErrorInvalidValue;
+  p.n_items = (int)items;
   p.scale_log2 = a.scale * kLog2e;
   p.causal = a.causal;
   p.o_bf16 = a.o_bf16;
   auto kern = prefill_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.Hq, a.B, p.n_qblocks);
+  // persistent: one CTA per SM (each owns all 512 TMEM columns)
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const int grid = p.n_items < sms ? p.n_items : sms;
   kern<<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
