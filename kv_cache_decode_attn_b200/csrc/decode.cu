@@ -222,7 +222,35 @@ __global__ void __launch_bounds__(DecodeCfg<D, MT>::kThreads, DecodeCfg<D, MT>::
       }
     }
 
-    // ---- online softmax (base-2 exponent, scale folded in)
+    // ---- V fragments for this warp's 16 tokens, loaded before the softmax so the
+    //      shared-memory latency overlaps it; keys at or past L may hold anything
+    //      (even NaN), so their V rows are zeroed
+    uint32_t vb[D / 16][4];
+    {
+      const bool tail = tok_base + 16 > L;
+      const int vrow = wsub * 16 + (lm & 1) * 8 + lr;
+      const int ta = tok_base + tig * 2, tb = ta + 8;
+      const uint32_t keep_a = ((ta < L) ? 0x0000ffffu : 0u) | ((ta + 1 < L) ? 0xffff0000u : 0u);
+      const uint32_t keep_b = ((tb < L) ? 0x0000ffffu : 0u) | ((tb + 1 < L) ? 0xffff0000u : 0u);
+#pragma unroll
+      for (int nn = 0; nn < D / 16; ++nn) {
+        const int chunk16 = nn * 2 + (lm >> 1);
+        const int h = chunk16 >> 3, cw = chunk16 & 7;
+        const uint32_t addr = vbase + h * C::kHalfBytes + vrow * 128 + ((cw ^ (vrow & 7)) << 4);
+        ldsm_x4_t(addr, vb[nn][0], vb[nn][1], vb[nn][2], vb[nn][3]);
+        if (tail) {
+          vb[nn][0] &= keep_a;
+          vb[nn][2] &= keep_a;
+          vb[nn][1] &= keep_b;
+          vb[nn][3] &= keep_b;
+        }
+      }
+    }
+
+    // ---- online softmax (base-2 exponent, scale folded in).  A row's reference
+    //      maximum is raised only when the tile maximum exceeds it by more than 8,
+    //      so O is rescaled rarely; p = 2^(s - m) then stays <= 256, and the merge
+    //      at the end uses the same reference, so the result is exact.
     float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
     for (int n = 0; n < 2; ++n) {
@@ -239,12 +267,24 @@ __global__ void __launch_bounds__(DecodeCfg<D, MT>::kThreads, DecodeCfg<D, MT>::
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-    const float mu0 = (mn0 == -INFINITY) ? 0.f : mn0;
-    const float mu1 = (mn1 == -INFINITY) ? 0.f : mn1;
-    const float al0 = ex2(m0 - mu0), al1 = ex2(m1 - mu1);
-    m0 = mn0;
-    m1 = mn1;
+    if (__any_sync(0xffffffffu, mx0 > m0 + 8.f || mx1 > m1 + 8.f)) {
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      const float al0 = ex2(m0 - ((mn0 == -INFINITY) ? 0.f : mn0));   // 0 while m is -inf
+      const float al1 = ex2(m1 - ((mn1 == -INFINITY) ? 0.f : mn1));
+      m0 = mn0;
+      m1 = mn1;
+      l0 *= al0;
+      l1 *= al1;
+#pragma unroll
+      for (int n = 0; n < D / 8; ++n) {
+        o_acc[n][0] *= al0;
+        o_acc[n][1] *= al0;
+        o_acc[n][2] *= al1;
+        o_acc[n][3] *= al1;
+      }
+    }
+    const float mu0 = (m0 == -INFINITY) ? 0.f : m0;
+    const float mu1 = (m1 == -INFINITY) ? 0.f : m1;
     float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
     for (int n = 0; n < 2; ++n) {
@@ -255,42 +295,19 @@ __global__ void __launch_bounds__(DecodeCfg<D, MT>::kThreads, DecodeCfg<D, MT>::
       ps0 += sacc[n][0] + sacc[n][1];
       ps1 += sacc[n][2] + sacc[n][3];
     }
-    l0 = l0 * al0 + ps0;
-    l1 = l1 * al1 + ps1;
-#pragma unroll
-    for (int n = 0; n < D / 8; ++n) {
-      o_acc[n][0] *= al0;
-      o_acc[n][1] *= al0;
-      o_acc[n][2] *= al1;
-      o_acc[n][3] *= al1;
-    }
+    l0 += ps0;
+    l1 += ps1;
     uint32_t pa[4];
     pa[0] = pack_bf16x2(sacc[0][0], sacc[0][1]);
     pa[1] = pack_bf16x2(sacc[0][2], sacc[0][3]);
     pa[2] = pack_bf16x2(sacc[1][0], sacc[1][1]);
     pa[3] = pack_bf16x2(sacc[1][2], sacc[1][3]);
 
-    // ---- O += P V ; keys at or past L may hold anything (even NaN): zero them
-    const bool tail = tok_base + 16 > L;
-    const int vrow = wsub * 16 + (lm & 1) * 8 + lr;
+    // ---- O += P V
 #pragma unroll
     for (int nn = 0; nn < D / 16; ++nn) {
-      const int chunk16 = nn * 2 + (lm >> 1);
-      const int h = chunk16 >> 3, cw = chunk16 & 7;
-      const uint32_t addr = vbase + h * C::kHalfBytes + vrow * 128 + ((cw ^ (vrow & 7)) << 4);
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4_t(addr, b0, b1, b2, b3);
-      if (tail) {
-        const int ta = tok_base + tig * 2, tb = ta + 8;
-        const uint32_t mlo_a = (ta < L) ? 0x0000ffffu : 0u, mhi_a = (ta + 1 < L) ? 0xffff0000u : 0u;
-        const uint32_t mlo_b = (tb < L) ? 0x0000ffffu : 0u, mhi_b = (tb + 1 < L) ? 0xffff0000u : 0u;
-        b0 &= (mlo_a | mhi_a);
-        b2 &= (mlo_a | mhi_a);
-        b1 &= (mlo_b | mhi_b);
-        b3 &= (mlo_b | mhi_b);
-      }
-      mma_bf16_16816(o_acc[2 * nn], pa, b0, b1);
-      mma_bf16_16816(o_acc[2 * nn + 1], pa, b2, b3);
+      mma_bf16_16816(o_acc[2 * nn], pa, vb[nn][0], vb[nn][1]);
+      mma_bf16_16816(o_acc[2 * nn + 1], pa, vb[nn][2], vb[nn][3]);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
