@@ -129,7 +129,8 @@ ATTN_API size_t attn_decode_workspace_bytes(int B, int T, int Hq, int Hkv, int d
  *               into at most n chunks
  *   workspace   device memory of at least attn_decode_workspace_bytes(...) bytes,
  *               16-byte aligned; contents on entry do not matter
- * Rows per KV head (Hq / Hkv) * T must be <= 32.
+ * Rows per KV head R = (Hq / Hkv) * T must be <= 128: R <= 32 runs on warp-level
+ * MMAs, 33 <= R <= 128 on the tcgen05 tensor cores with the scores in TMEM.
  * Errors: ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED (d, rows per KV head),
  * ATTN_ERR_WORKSPACE, ATTN_ERR_CUDA.  Bad lengths or page ids found on the
  * device set ATTN_DEV_SEQLEN / ATTN_DEV_PAGE_ID and make the affected rows NaN.

@@ -202,7 +202,7 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
   if (max_seqlen_k == 0) max_seqlen_k = capacity_tokens;
   if (max_seqlen_k < T || max_seqlen_k > capacity_tokens) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-  if ((Hq / Hkv) * T > 32) return ATTN_ERR_UNSUPPORTED;
+  if ((Hq / Hkv) * T > 128) return ATTN_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
   DecodeLayout L;
   if (!decode_layout(B, T, Hq, Hkv, d, max_seqlen_k, num_splits, &L)) return ATTN_ERR_INVALID_ARG;

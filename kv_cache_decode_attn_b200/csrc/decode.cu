@@ -128,11 +128,19 @@ __global__ void __launch_bounds__(DecodeCfg<D, MT>::kThreads, DecodeCfg<D, MT>::
             tma_load_3d(vst + h * C::kHalfBytes, &tmV, &full[s], h * 64, g, row, pol);
           }
         } else {
-          const int nb = min(kDecodeTile / kPageTokens, (tok_end - t0 + kPageTokens - 1) / kPageTokens);
-          mbar_arrive_expect_tx(&full[s], nb * 2 * C::kHalves * kPageTokens * 128);
+          constexpr int kBlocks = kDecodeTile / kPageTokens;
+          const int nb = min(kBlocks, (tok_end - t0 + kPageTokens - 1) / kPageTokens);
           const int32_t* row_tab = p.page_table + (size_t)b * p.max_blocks + t0 / kPageTokens;
-          for (int j = 0; j < nb; ++j) {
-            int blk = row_tab[j];
+          // read the stage's block ids together: the copies' memory clobbers would
+          // otherwise serialise one table read per block
+          int ids[kBlocks];
+#pragma unroll
+          for (int j = 0; j < kBlocks; ++j) ids[j] = j < nb ? __ldg(row_tab + j) : 0;
+          mbar_arrive_expect_tx(&full[s], nb * 2 * C::kHalves * kPageTokens * 128);
+#pragma unroll
+          for (int j = 0; j < kBlocks; ++j) {
+            if (j >= nb) break;
+            int blk = ids[j];
             if (blk < 0 || blk >= p.num_blocks) {
               atomicOr(p.status, DEV_PAGE_ID);
               blk = 0;   // keep the byte count; the result is flagged invalid
@@ -503,12 +511,16 @@ int decode_chunk_tokens(int B, int Hkv, int rows, int max_seqlen, int num_splits
   if (num_splits > 0) {
     chunk = (max_seqlen + num_splits - 1) / num_splits;
   } else {
-    chunk = rows <= 8 ? 512 : (rows <= 16 ? 1024 : 2048);
-    // short caches: keep at least ~2 work items per SM
-    while (chunk > 256 && (long long)B * Hkv * ((max_seqlen + chunk - 1) / chunk) < 296) chunk >>= 1;
+    // Long chunks stream longer and leave fewer partials to merge; measured on
+    // B200 the best were 2048 tokens for 16 x 8 sequence-heads up to 32K keys and
+    // 4096 for 8 x 8 up to 128K.  Start at 4096 and halve until the grid holds
+    // about 14 work items per SM (counted as if every sequence had max_seqlen).
+    chunk = 4096;
+    while (chunk > 256 && (long long)B * Hkv * ((max_seqlen + chunk - 1) / chunk) < 2048) chunk >>= 1;
   }
-  chunk = ((chunk + kDecodeTile - 1) / kDecodeTile) * kDecodeTile;
-  return chunk < kDecodeTile ? kDecodeTile : chunk;
+  // a multiple of both kernels' tiles
+  chunk = ((chunk + kDecodeTcTile - 1) / kDecodeTcTile) * kDecodeTcTile;
+  return chunk < kDecodeTcTile ? kDecodeTcTile : chunk;
 }
 
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
@@ -537,7 +549,8 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
 
   // K/V viewed as 3-D {d, Hkv, rows}: rows = B * capacity (contiguous) or num_blocks * 16 (paged)
   const uint64_t rows = paged ? (uint64_t)a.num_blocks * kPageTokens : (uint64_t)a.B * a.capacity;
-  const uint32_t box_rows = paged ? kPageTokens : kDecodeTile;
+  const bool tc = R > kDecodeMmaRows;
+  const uint32_t box_rows = paged ? kPageTokens : (tc ? kDecodeTcTile : kDecodeTile);
   CUtensorMap tk, tv;
   const uint64_t s1 = (uint64_t)a.d * 2, s2 = (uint64_t)a.Hkv * a.d * 2;
   if (encode_tmap_3d(&tk, a.k, a.d, a.Hkv, rows, s1, s2, 64, 1, box_rows) ||
@@ -545,7 +558,9 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
     return cudaErrorInvalidValue;
 
   cudaError_t e;
-  if (a.d == 128) {
+  if (tc) {
+    e = launch_decode_tc(a, tk, tv, stream);
+  } else if (a.d == 128) {
     if (R <= 16) e = paged ? run_split<128, 1, true>(tk, tv, sp, a.B, stream) : run_split<128, 1, false>(tk, tv, sp, a.B, stream);
     else e = paged ? run_split<128, 2, true>(tk, tv, sp, a.B, stream) : run_split<128, 2, false>(tk, tv, sp, a.B, stream);
   } else {

@@ -1,0 +1,439 @@
+// Split-KV decode attention on the sm_100a tensor cores, for many query rows per
+// KV head (R = (Hq/Hkv) * T from 33 to 128: grouped heads times several new
+// tokens, e.g. a speculative-verify step of 8 or 16 tokens).
+//
+// One CTA owns one work item (key chunk c, KV head g, sequence b), exactly like
+// the warp-MMA decode kernel, and writes the same per-chunk partials (normalised
+// O and log-sum-exp per row) that the combine kernel merges.  The R query rows
+// of KV head g form one 128-row tcgen05 tile (row r = t * G + hh; rows >= R are
+// zero).  Warp roles:
+//   warps 0..3  softmax: thread i owns row i (TMEM lane i); warps whose rows are
+//               all >= R stay idle;
+//   warp 4      TMA producer: Q once, then 128-token K/V tiles (contiguous: one
+//               128-row box per 64 columns of d; paged: one 16-row box per
+//               physical block, its page-table entry checked first) into a
+//               2-stage ring with the evict-first L2 policy;
+//   warp 5      MMA issuer: S_j = Q K_j^T (SS) into one of two TMEM S buffers,
+//               O += P_j V_j (P read from TMEM, where the softmax wrote it over
+//               the consumed S columns).  S_{j+1} is issued before PV_j, so the
+//               tensor core computes the next scores while the softmax runs.
+// Online softmax with the lazy rescale of the prefill kernel: a row's reference
+// maximum is raised only when a tile's maximum exceeds it by more than 8.
+//
+// Method: "[BEE-30062] FlashAttention 與高效注意力核心", "背景" and
+// "為長上下文推論啟用 FlashDecoding" (split along the KV length, stable merge of
+// partial softmax results); "Effizienz", "Der wichtige Maskenfehler beim Cache"
+// (several new tokens need the positional offset in the mask); "大模型面試笔记"
+// section 2 (online safe softmax).
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace kvattn {
+namespace {
+
+constexpr int kRows = 128;   // MMA M (query rows per KV head, padded)
+constexpr int kTok = 128;    // keys per K/V tile
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+template <int D>
+struct TcCfg {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kHalfBytes = kTok * 128;              // 128 rows x 128 B
+  static constexpr int kTileBytes = kTok * D * 2;            // one K or V tile (= the Q tile)
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kQOff + kTileBytes;           // K stages 0, 1
+  static constexpr int kVOff = kKOff + 2 * kTileBytes;       // V stages 0, 1
+  static constexpr int kBarOff = kVOff + 2 * kTileBytes;
+  static constexpr int kSmemBytes = kBarOff + 256 + 1024;
+  static constexpr int kTmemCols = 512;                      // S0 | S1 | O (+ unused)
+  static constexpr int kOCol = 256;
+};
+
+// K and V stages are released separately: K_j as soon as S_j is done, V_j once PV_j is done.
+// P_FULL is one barrier per S buffer: S_{j+1} exists before PV_j is issued, so a
+// fast softmax warp may finish tile j+1 while a slow one is still on tile j, and
+// its arrival must not count towards tile j.
+// O_DONE completes once per PV and is waited on only one tile behind (before a
+// rescale, where PV_{j-2} is known to be done); the epilogue, which may be two
+// PVs behind, waits on O_FINAL, committed once after the last PV.
+enum TcBar { T_Q = 0, T_KFULL = 1, T_VFULL = 3, T_KEMPTY = 5, T_VEMPTY = 7, T_SFULL = 9, T_PFULL = 11, T_ODONE = 13,
+             T_OFINAL = 14, T_DRAIN = 15, T_COUNT = 16 };
+
+struct TcParams {
+  const int32_t* seqlens;
+  const int32_t* page_table;
+  float* part_o;
+  float* part_lse;
+  unsigned* status;
+  int T, Hq, Hkv, G, R;
+  int chunk, max_chunks, capacity, max_blocks, num_blocks, max_seqlen;
+  float scale_log2;
+  int causal;
+};
+
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                        unsigned* status) {
+  if (*abort_flag) return false;
+  if (mbar_wait(bar, parity)) return true;
+  atomicOr(status, DEV_TIMEOUT);
+  *abort_flag = 1;
+  return false;
+}
+
+template <int D, bool PAGED>
+__global__ void __launch_bounds__(192, 1)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const TcParams p) {
+  using C = TcCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + T_COUNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int L = p.seqlens[b];
+  // invalid lengths are reported (and their rows made NaN) by the combine kernel
+  if (L < p.T || L > p.max_seqlen || (!PAGED && L > p.capacity) ||
+      (PAGED && (L + kPageTokens - 1) / kPageTokens > p.max_blocks))
+    return;
+  const int tok_begin = c * p.chunk;
+  if (tok_begin >= L) return;
+  const int tok_end = min(tok_begin + p.chunk, L);
+  const int n_tiles = (tok_end - tok_begin + kTok - 1) / kTok;
+  const int active_warps = (p.R + 31) / 32;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[T_Q], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars[T_KFULL + s], 1);
+      mbar_init(&bars[T_VFULL + s], 1);
+      mbar_init(&bars[T_KEMPTY + s], 1);
+      mbar_init(&bars[T_VEMPTY + s], 1);
+      mbar_init(&bars[T_SFULL + s], 1);
+      mbar_init(&bars[T_PFULL + s], active_warps);
+    }
+    mbar_init(&bars[T_ODONE], 1);
+    mbar_init(&bars[T_OFINAL], 1);
+    mbar_init(&bars[T_DRAIN], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  // rows R..127 of the Q tile are never loaded: make them zero (whole 128-byte rows)
+  {
+    const int per_half = (kRows - p.R) * 8;   // 16-byte chunks of rows R..127 in one half of d
+    for (int i = threadIdx.x; i < per_half * C::kHalves; i += blockDim.x) {
+      const int half = i / per_half, rem = i - half * per_half;
+      *reinterpret_cast<uint4*>(smem + C::kQOff + half * C::kHalfBytes + p.R * 128 + rem * 16) =
+          make_uint4(0, 0, 0, 0);
+    }
+  }
+  fence_proxy_async_smem();
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      const uint64_t pol = policy_evict_first();
+      // Q rows (t, head g*G + hh) for t < T, hh < G: one box {64, G, T, 1} per half of d
+      mbar_arrive_expect_tx(&bars[T_Q], p.R * D * 2);
+#pragma unroll
+      for (int hh = 0; hh < C::kHalves; ++hh)
+        tma_load_4d(smem + C::kQOff + hh * C::kHalfBytes, &tmQ, &bars[T_Q], hh * 64, g * p.G, 0, b, pol);
+      int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};
+      constexpr int kBlocks = kTok / kPageTokens;
+      // physical blocks of one tile, read together (the copies' memory clobbers
+      // would otherwise serialise one table read per block)
+      auto read_ids = [&](int i, int (&ids)[kBlocks]) {
+        const int t0 = tok_begin + i * kTok;
+        const int nb = min(kBlocks, (tok_end - t0 + kPageTokens - 1) / kPageTokens);
+        const int32_t* tab = p.page_table + (size_t)b * p.max_blocks + t0 / kPageTokens;
+#pragma unroll
+        for (int j = 0; j < kBlocks; ++j) ids[j] = j < nb ? __ldg(tab + j) : 0;
+#pragma unroll
+        for (int j = 0; j < kBlocks; ++j)
+          if (j < nb && (ids[j] < 0 || ids[j] >= p.num_blocks)) {
+            atomicOr(p.status, DEV_PAGE_ID);
+            ids[j] = 0;   // keep the byte count; the result is flagged invalid
+          }
+        return nb;
+      };
+      // one tensor (K or V) of tile i into ring stage i & 1
+      auto load = [&](const CUtensorMap* map, uint8_t* base, uint64_t* full, int i, const int (&ids)[kBlocks],
+                      int nb) {
+        const int t0 = tok_begin + i * kTok;
+        if (!PAGED) {
+          mbar_arrive_expect_tx(full, C::kTileBytes);
+#pragma unroll
+          for (int hh = 0; hh < C::kHalves; ++hh)
+            tma_load_3d(base + hh * C::kHalfBytes, map, full, hh * 64, g, b * p.capacity + t0, pol);
+        } else {
+          mbar_arrive_expect_tx(full, nb * C::kHalves * kPageTokens * 128);
+#pragma unroll
+          for (int j = 0; j < kBlocks; ++j) {
+            if (j >= nb) break;
+#pragma unroll
+            for (int hh = 0; hh < C::kHalves; ++hh)
+              tma_load_3d(base + hh * C::kHalfBytes + j * kPageTokens * 128, map, full, hh * 64, g,
+                          ids[j] * kPageTokens, pol);
+          }
+        }
+      };
+      int ids[kBlocks] = {0, 0, 0, 0, 0, 0, 0, 0};
+      int nb = PAGED ? read_ids(0, ids) : 0;
+      for (int i = 0; i < n_tiles; ++i) {
+        const int st = i & 1;
+        if (i >= 2 && !tc_wait(&bars[T_KEMPTY + st], ((i >> 1) - 1) & 1, abort_flag, p.status)) break;
+        last_k[st] = i;
+        load(&tmK, smem + C::kKOff + st * C::kTileBytes, &bars[T_KFULL + st], i, ids, nb);
+        if (i >= 2 && !tc_wait(&bars[T_VEMPTY + st], ((i >> 1) - 1) & 1, abort_flag, p.status)) break;
+        last_v[st] = i;
+        load(&tmV, smem + C::kVOff + st * C::kTileBytes, &bars[T_VFULL + st], i, ids, nb);
+        if (PAGED && i + 1 < n_tiles) nb = read_ids(i + 1, ids);
+      }
+      // no copy may still be landing in shared memory when the CTA exits
+      mbar_wait(&bars[T_Q], 0);
+      for (int st = 0; st < 2; ++st) {
+        if (last_k[st] >= 0) mbar_wait(&bars[T_KFULL + st], (last_k[st] >> 1) & 1);
+        if (last_v[st] >= 0) mbar_wait(&bars[T_VFULL + st], (last_v[st] >> 1) & 1);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(kRows, kTok, 0, 0);
+      constexpr uint32_t idO = idesc_bf16(kRows, D, 0, 1);
+      const uint32_t q_s = smem_u32(smem + C::kQOff);
+      auto issue_s = [&](int i) {
+        const int st = i & 1;
+        const uint32_t k_s = smem_u32(smem + C::kKOff + st * C::kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
+          tc_mma_ss(tmem + st * 128, smem_desc(q_s + off, 16, 1024), smem_desc(k_s + off, 16, 1024), idS, kk > 0);
+        }
+        tc_commit(&bars[T_SFULL + st]);
+        tc_commit(&bars[T_KEMPTY + st]);     // K_i is read only by S_i
+      };
+      bool ok = tc_wait(&bars[T_Q], 0, abort_flag, p.status) &&
+                tc_wait(&bars[T_KFULL], 0, abort_flag, p.status);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+      }
+      for (int i = 0; ok && i < n_tiles; ++i) {
+        const int st = i & 1;
+        if (i + 1 < n_tiles) {
+          ok = tc_wait(&bars[T_KFULL + ((i + 1) & 1)], ((i + 1) >> 1) & 1, abort_flag, p.status);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(i + 1);   // its S buffer last held P_{i-1}, whose PV was issued before
+        }
+        ok = tc_wait(&bars[T_PFULL + st], (i >> 1) & 1, abort_flag, p.status) &&
+             tc_wait(&bars[T_VFULL + st], (i >> 1) & 1, abort_flag, p.status);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t v_s = smem_u32(smem + C::kVOff + st * C::kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < kTok / 16; ++kk)
+          tc_mma_ts(tmem + C::kOCol, tmem + st * 128 + kk * 8, smem_desc(v_s + kk * 16 * 128, C::kHalfBytes, 1024),
+                    idO, (i > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&bars[T_ODONE]);
+        tc_commit(&bars[T_VEMPTY + st]);
+      }
+      // also on a failed wait, so that the epilogue does not wait in vain (abort_flag marks the result)
+      tc_commit(&bars[T_OFINAL]);
+    }
+  } else if (warp < active_warps) {
+    // ------------------------------------------------------------- softmax warps
+    const int row = warp * 32 + lane;
+    const bool live = row < p.R;
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const int t = live ? row / p.G : 0;
+    const int end = p.causal ? L - p.T + t + 1 : L;       // first invisible key of this row
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int i = 0; i < n_tiles; ++i) {
+      const int st = i & 1;
+      if (!tc_wait(&bars[T_SFULL + st], (i >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t s_addr = lane_base + st * 128;
+      float s[kTok];
+#pragma unroll
+      for (int cc = 0; cc < kTok; cc += 32) {
+        uint32_t r[32];
+        tmem_ld32(s_addr + cc, r);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) s[cc + e] = __uint_as_float(r[e]);
+      }
+      tc_wait_ld();
+      const int key0 = tok_begin + i * kTok;
+      const int lim = live ? end - key0 : 0;              // visible keys of this row in the tile: [0, lim)
+      if (lim < kTok) {
+#pragma unroll
+        for (int cc = 0; cc < kTok; ++cc) s[cc] = (cc < lim) ? s[cc] : -INFINITY;
+      }
+      float mx8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx8[k] = max3f(s[k], s[k + 8], s[k + 16]);
+#pragma unroll
+      for (int cc = 24; cc + 8 < kTok; cc += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx8[k] = max3f(mx8[k], s[cc + k], s[cc + 8 + k]);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], s[kTok - 8 + k]);
+      float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+      mx *= p.scale_log2;
+      const bool warp_raise = __any_sync(0xffffffffu, mx > m + 8.f);
+      float alpha = 1.f;
+      if (warp_raise) {
+        const float m_new = fmaxf(m, mx);
+        alpha = ex2(m - ((m_new == -INFINITY) ? 0.f : m_new));   // 0 while m is -inf
+        m = m_new;
+      }
+      const float neg_mu = (m == -INFINITY) ? 0.f : -m;
+      float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int cc = 0; cc < kTok; cc += 16) {
+        uint32_t pk[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          const float p0 = ex2(fmaf(s[cc + e], p.scale_log2, neg_mu));
+          const float p1 = ex2(fmaf(s[cc + e + 1], p.scale_log2, neg_mu));
+          ls4[(e >> 1) & 3] += p0 + p1;
+          pk[e / 2] = pack_bf16x2(p0, p1);
+        }
+        tmem_st8(s_addr + cc / 2, pk);      // P row over the consumed S columns
+      }
+      l = l * alpha + ((ls4[0] + ls4[1]) + (ls4[2] + ls4[3]));
+      if (warp_raise && i > 0) {
+        // PV_{i-1} must be done before O is rescaled (S_i was issued before it)
+        if (!tc_wait(&bars[T_ODONE], (i - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int cc = 0; cc < D; cc += 32) {
+          uint32_t r[32];
+          tmem_ld32(lane_base + C::kOCol + cc, r);
+          tc_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tmem_st32(lane_base + C::kOCol + cc, r);
+        }
+      }
+      // keys at or past L may hold anything (even NaN): zero their V rows, which
+      // the PV MMA would otherwise multiply by p = 0
+      const int valid = L - key0;
+      if (valid < kTok && warp == 0) {
+        if (!tc_wait(&bars[T_VFULL + st], (i >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+        uint8_t* vst = smem + C::kVOff + st * C::kTileBytes;
+        for (int idx = max(valid, 0) * 8 + lane; idx < kTok * 8; idx += 32)
+#pragma unroll
+          for (int hh = 0; hh < C::kHalves; ++hh)
+            *reinterpret_cast<uint4*>(vst + hh * C::kHalfBytes + idx * 16) = make_uint4(0, 0, 0, 0);
+        fence_proxy_async_smem();
+      }
+      tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[T_PFULL + st]);
+    }
+
+    // ---------------------------------------------------------- epilogue
+    if (ok && tc_wait(&bars[T_OFINAL], 0, abort_flag, p.status) && !*abort_flag) {
+      tc_fence_after();
+      const size_t item = ((size_t)b * p.Hkv + g) * p.max_chunks + c;
+      float* out = p.part_o + (item * p.R + row) * D;
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+      for (int cc = 0; cc < D; cc += 32) {
+        uint32_t r[32];
+        tmem_ld32(lane_base + C::kOCol + cc, r);
+        tc_wait_ld();
+        if (live) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(out + cc + e) =
+                make_float4(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l,
+                            __uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
+        }
+      }
+      if (live) p.part_lse[item * p.R + row] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+    } else if (live) {
+      p.part_lse[(((size_t)b * p.Hkv + g) * p.max_chunks + c) * p.R + row] = NAN;   // a wait gave up
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && warp == 5 && lane == 0) {
+    tc_commit(&bars[T_DRAIN]);
+    mbar_wait(&bars[T_DRAIN], 0);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int D, bool PAGED>
+cudaError_t run_tc(const DecodeLaunch& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream) {
+  using C = TcCfg<D>;
+  const int G = a.Hq / a.Hkv;
+  CUtensorMap tq;
+  // q [B, T, Hq, d] as {d, Hq, T, B}; one box covers the G heads of a KV head for every new token
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)a.Hq, (cuuint64_t)a.T, (cuuint64_t)a.B};
+  cuuint64_t str[3] = {(cuuint64_t)D * 2, (cuuint64_t)a.Hq * D * 2, (cuuint64_t)a.T * a.Hq * D * 2};
+  cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)a.T, 1};
+  if (encode_tmap_nd(&tq, a.q, 4, dims, str, box)) return cudaErrorInvalidValue;
+  TcParams p;
+  p.seqlens = a.seqlens;
+  p.page_table = a.page_table;
+  p.part_o = a.part_o;
+  p.part_lse = a.part_lse;
+  p.status = a.status;
+  p.T = a.T;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.G = G;
+  p.R = G * a.T;
+  p.chunk = a.chunk;
+  p.max_chunks = a.max_chunks;
+  p.capacity = a.capacity;
+  p.max_blocks = a.max_blocks;
+  p.num_blocks = a.num_blocks;
+  p.max_seqlen = a.max_seqlen;
+  p.scale_log2 = a.scale * kLog2e;
+  p.causal = a.causal;
+  auto kern = decode_tc_kernel<D, PAGED>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.max_chunks, a.Hkv, a.B);
+  kern<<<grid, 192, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode_tc(const DecodeLaunch& a, const CUtensorMap& tk, const CUtensorMap& tv,
+                             cudaStream_t stream) {
+  const bool paged = a.page_table != nullptr;
+  if (a.d == 128) return paged ? run_tc<128, true>(a, tk, tv, stream) : run_tc<128, false>(a, tk, tv, stream);
+  return paged ? run_tc<64, true>(a, tk, tv, stream) : run_tc<64, false>(a, tk, tv, stream);
+}
+
+}  // namespace kvattn

@@ -9,7 +9,12 @@
 namespace kvattn {
 
 constexpr int kPageTokens = 16;   // tokens per physical KV block
-constexpr int kDecodeTile = 64;   // tokens per pipeline stage of the decode kernel
+constexpr int kDecodeTile = 64;   // tokens per pipeline stage of the warp-MMA decode kernel
+constexpr int kDecodeTcTile = 128;  // tokens per K/V tile of the tensor-core decode kernel
+// Above this many query rows per KV head the tensor-core kernel runs.  Up to 32
+// the warp-MMA kernel is faster: its four consumer warps use all four SM
+// sub-partitions, while the tensor-core kernel's rows all sit in one warp.
+constexpr int kDecodeMmaRows = 32;
 
 struct DecodeLaunch {
   const void* q;
@@ -70,6 +75,8 @@ int encode_tmap_3d(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t d
                    uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1, uint32_t box2);
 
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream);
+// tcgen05 split kernel for more than 16 query rows per KV head (K/V maps with 128-row boxes when contiguous)
+cudaError_t launch_decode_tc(const DecodeLaunch& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream);
 cudaError_t launch_append(const AppendLaunch& a, cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillLaunch& a, cudaStream_t stream);
 

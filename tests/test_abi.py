@@ -94,7 +94,7 @@ def test_decode_rejects_bad_arguments():
     assert call(T=4, msk=3) == kv.ATTN_ERR_INVALID_ARG        # fewer keys than new tokens
     assert call(pt=P, mb=0, nb=10) == kv.ATTN_ERR_INVALID_ARG
     assert call(d=80) == kv.ATTN_ERR_UNSUPPORTED
-    assert call(Hq=64, Hkv=1, T=1) == kv.ATTN_ERR_UNSUPPORTED   # 64 rows per KV head
+    assert call(Hq=64, Hkv=1, T=4) == kv.ATTN_ERR_UNSUPPORTED   # 256 rows per KV head
     assert call(ws=None) == kv.ATTN_ERR_WORKSPACE
     assert call(wsb=16) == kv.ATTN_ERR_WORKSPACE
     assert call(ns=-1) == kv.ATTN_ERR_INVALID_ARG

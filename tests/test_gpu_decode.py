@@ -81,6 +81,23 @@ def test_decode_small_parity(paged, T, Hq, Hkv, d):
     check_lse(lse, lse_ref)
 
 
+@pytest.mark.parametrize("paged", [False, True])
+@pytest.mark.parametrize("T,Hq,Hkv,d", [(5, 16, 4, 128), (8, 64, 8, 128), (16, 32, 4, 128), (6, 40, 5, 64),
+                                        (16, 8, 1, 64), (2, 128, 2, 128)])
+def test_decode_many_rows_per_kv_head(paged, T, Hq, Hkv, d):
+    """More than 16 query rows per KV head (grouped heads x new tokens, up to 128):
+    the tensor-core split kernel, with the positional-offset mask."""
+    lens = [0, 100, 127, 128, 129, 1000, 5000]
+    case = synth.decode_inputs(len(lens), T, Hq, Hkv, d, 0, 0, seed=300 + T * Hq + d, device="cuda", paged=paged,
+                               lengths=lens, spare_blocks=2)
+    host = host_copy(case)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = run_step(case, T, Hq, Hkv, d, scale)
+    o_ref, lse_ref = oracle_step(host, T, scale)
+    check_o(o, o_ref)
+    check_lse(lse, lse_ref)
+
+
 @pytest.mark.parametrize("num_splits", [1, 2, 3, 7, 40])
 @pytest.mark.parametrize("T", [1, 4])
 def test_decode_split_counts(num_splits, T):
@@ -122,6 +139,36 @@ def test_decode_ignores_nonfinite_past_the_end():
                 if slot0:
                     case.k_pool[last, slot0:] = float("nan")
                     case.v_pool[last, slot0:] = float("inf")
+        else:
+            for b, L in enumerate(lens):
+                case.k_cache[b, L + T:] = float("nan")
+                case.v_cache[b, L + T:] = float("nan")
+        host = host_copy(case)
+        o, lse = run_step(case, T, Hq, Hkv, d, 0.1)
+        o_ref, lse_ref = oracle_step(host, T, 0.1)
+        check_o(o, o_ref)
+        check_lse(lse, lse_ref)
+
+
+def test_decode_many_rows_ignores_nonfinite_past_the_end():
+    T, Hq, Hkv, d = 8, 32, 4, 128
+    lens = [3, 120, 300, 1021]
+    for paged in (False, True):
+        case = synth.decode_inputs(len(lens), T, Hq, Hkv, d, 0, 0, seed=19, device="cuda", paged=paged,
+                                   lengths=lens, capacity=1200, spare_blocks=2)
+        if paged:
+            for b, L in enumerate(lens):
+                nb = (L + T + 15) // 16
+                last = int(case.page_table[b, nb - 1])
+                slot0 = (L + T) % 16
+                if slot0:
+                    case.k_pool[last, slot0:] = float("nan")
+                    case.v_pool[last, slot0:] = float("inf")
+            used = set(int(x) for x in case.page_table.ravel() if x >= 0)
+            spare = [i for i in range(case.k_pool.shape[0]) if i not in used]
+            assert spare
+            case.k_pool[spare[0]] = float("nan")                     # a block no page-table entry references
+            case.v_pool[spare[-1]] = float("nan")
         else:
             for b, L in enumerate(lens):
                 case.k_cache[b, L + T:] = float("nan")
