@@ -38,3 +38,4 @@ from .kv_bytes import (  # noqa: F401
     max_concurrent_requests,
 )
 from . import selfcheck  # noqa: F401
+from . import fp8  # noqa: F401

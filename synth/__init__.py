@@ -16,6 +16,11 @@ Recipe (the same on every machine with the same torch build):
   block ids are a seeded random permutation of ``range(total blocks)``
   (NumPy's ``permutation``, a Fisher-Yates shuffle); unused page-table entries
   hold -1.
+* FP8 caches: per-KV-head float32 scales drawn uniformly from
+  ``[1/64, 1/16]`` (PCG64); the stored codes are PyTorch's own float8_e4m3fn
+  cast of seeded N(0, 1) draws divided by the head's scale (clamped to +-448),
+  so that the dequantised cache is again about N(0, 1).  The library's own
+  quantiser (the FP8 append path) is not involved in making inputs.
 * Seeds: ``1000 + index`` of the workload in ``WORKLOADS`` unless a test
   chooses its own.
 """
@@ -58,6 +63,7 @@ class Decode:
     len_hi: int
     paged: bool = False
     causal: bool = True
+    fp8: bool = False
 
     @property
     def scale(self) -> float:
@@ -75,6 +81,11 @@ WORKLOADS = {
                            paged=True),
     "decode_paged_t4": Decode("decode_paged_t4", B=8, T=4, Hq=64, Hkv=8, d=128, len_lo=32768,
                               len_hi=131072, paged=True),
+    # the same decode steps over an FP8 (e4m3) cache with per-KV-head scales
+    "decode_contig_fp8": Decode("decode_contig_fp8", B=16, T=1, Hq=32, Hkv=8, d=128, len_lo=1024,
+                                len_hi=32768, fp8=True),
+    "decode_paged_fp8": Decode("decode_paged_fp8", B=8, T=1, Hq=64, Hkv=8, d=128, len_lo=32768,
+                               len_hi=131072, paged=True, fp8=True),
 }
 
 SEEDS = {name: 1000 + i for i, name in enumerate(WORKLOADS)}
@@ -85,6 +96,23 @@ def normal_bf16(shape, seed: int, device="cpu") -> torch.Tensor:
     g = torch.Generator(device=device)
     g.manual_seed(int(seed))
     return torch.randn(tuple(shape), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+
+
+def kv_scales(Hkv: int, seed: int) -> np.ndarray:
+    """Per-KV-head float32 scales, uniform on ``[1/64, 1/16]``."""
+    rng = np.random.Generator(np.random.PCG64(int(seed)))
+    return rng.uniform(1.0 / 64, 1.0 / 16, size=Hkv).astype(np.float32)
+
+
+def normal_e4m3_codes(shape, scales: np.ndarray, seed: int, device="cpu") -> torch.Tensor:
+    """uint8 e4m3 codes of N(0, 1) / scale[head] (head = second-to-last axis),
+    made by PyTorch's float8_e4m3fn cast."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    x = torch.randn(tuple(shape), generator=g, device=device, dtype=torch.float32)
+    inv = torch.as_tensor(1.0 / np.asarray(scales, dtype=np.float64), dtype=torch.float32, device=device)
+    x = (x * inv[:, None]).clamp(-448.0, 448.0)
+    return x.to(torch.float8_e4m3fn).view(torch.uint8)
 
 
 def uniform_lengths(B: int, lo: int, hi: int, seed: int) -> np.ndarray:
@@ -120,20 +148,28 @@ class DecodeCase:
     k_pool: torch.Tensor | None = None      # paged [num_blocks, 16, Hkv, d]
     v_pool: torch.Tensor | None = None
     page_table: np.ndarray | None = None    # int32 [B, max_blocks], -1 = unused
+    k_scale: np.ndarray | None = None       # FP8 caches: float32 [Hkv] per-KV-head scales
+    v_scale: np.ndarray | None = None
     extra: dict = field(default_factory=dict)
 
     @property
     def paged(self) -> bool:
         return self.page_table is not None
 
+    @property
+    def fp8(self) -> bool:
+        return self.k_scale is not None
+
 
 def decode_inputs(B, T, Hq, Hkv, d, len_lo, len_hi, seed, device="cpu", paged=False,
-                  lengths=None, capacity=None, spare_blocks=0) -> DecodeCase:
+                  lengths=None, capacity=None, spare_blocks=0, fp8=False) -> DecodeCase:
     """Cache contents, new tokens and queries for one decode step.
 
     ``lengths`` overrides the seeded cache lengths.  ``capacity`` sets the
     contiguous cache's token capacity (default ``max(lengths) + T``).  Paged
-    pools get ``spare_blocks`` extra unused blocks.
+    pools get ``spare_blocks`` extra unused blocks.  With ``fp8`` the cache
+    holds uint8 e4m3 codes and the case carries per-KV-head scales; the new
+    tokens stay bfloat16.
     """
     cache_lens = (np.asarray(lengths, dtype=np.int64) if lengths is not None
                   else uniform_lengths(B, len_lo, len_hi, seed))
@@ -142,10 +178,19 @@ def decode_inputs(B, T, Hq, Hkv, d, len_lo, len_hi, seed, device="cpu", paged=Fa
     k_new = normal_bf16((B, T, Hkv, d), seed * 7 + 1, device)
     v_new = normal_bf16((B, T, Hkv, d), seed * 7 + 2, device)
     case = DecodeCase(q=q, k_new=k_new, v_new=v_new, cache_lens=cache_lens, seqlens_k=seqlens_k)
+    if fp8:
+        case.k_scale = kv_scales(Hkv, seed * 7 + 6)
+        case.v_scale = kv_scales(Hkv, seed * 7 + 7)
+
+    def values(shape, s, which):
+        if fp8:
+            return normal_e4m3_codes(shape, case.k_scale if which == 0 else case.v_scale, s, device)
+        return normal_bf16(shape, s, device)
+
     if not paged:
         cap = int(capacity) if capacity is not None else int(seqlens_k.max())
-        case.k_cache = normal_bf16((B, cap, Hkv, d), seed * 7 + 3, device)
-        case.v_cache = normal_bf16((B, cap, Hkv, d), seed * 7 + 4, device)
+        case.k_cache = values((B, cap, Hkv, d), seed * 7 + 3, 0)
+        case.v_cache = values((B, cap, Hkv, d), seed * 7 + 4, 1)
         return case
     nblk = [(int(L) + PAGE_TOKENS - 1) // PAGE_TOKENS for L in seqlens_k]
     total = sum(nblk) + int(spare_blocks)
@@ -157,8 +202,8 @@ def decode_inputs(B, T, Hq, Hkv, d, len_lo, len_hi, seed, device="cpu", paged=Fa
         table[b, :nblk[b]] = perm[off:off + nblk[b]]
         off += nblk[b]
     case.page_table = table
-    case.k_pool = normal_bf16((total, PAGE_TOKENS, Hkv, d), seed * 7 + 3, device)
-    case.v_pool = normal_bf16((total, PAGE_TOKENS, Hkv, d), seed * 7 + 4, device)
+    case.k_pool = values((total, PAGE_TOKENS, Hkv, d), seed * 7 + 3, 0)
+    case.v_pool = values((total, PAGE_TOKENS, Hkv, d), seed * 7 + 4, 1)
     return case
 
 
@@ -170,4 +215,4 @@ def workload_prefill(name: str, device="cpu"):
 def workload_decode(name: str, device="cpu", **kw) -> tuple[Decode, DecodeCase]:
     w = WORKLOADS[name]
     return w, decode_inputs(w.B, w.T, w.Hq, w.Hkv, w.d, w.len_lo, w.len_hi, SEEDS[name],
-                            device=device, paged=w.paged, **kw)
+                            device=device, paged=w.paged, fp8=w.fp8, **kw)
