@@ -46,6 +46,11 @@ WORKLOAD_SETS = {
     "llama8b_layer": ("prefill_llama8b", "decode_contig"),
     "gpt2_prefill_paged_decode": ("prefill_gpt2", "decode_paged"),
     "llama8b_nc_paged_t4": ("prefill_llama8b_nc", "decode_paged_t4"),
+    # the same layer with an FP8 (e4m3, per-KV-head scales) KV cache
+    "llama8b_layer_fp8": ("prefill_llama8b", "decode_contig_fp8"),
+    "llama8b_paged_fp8": ("prefill_llama8b", "decode_paged_fp8"),
+    # prefill against an existing cache: 512-token prompt chunks on cached 4K..16K prefixes
+    "llama8b_chunked_prefill": ("prefill_llama8b", "prefill_chunk_paged"),
 }
 DEFAULT_SET = "llama8b_layer"
 
@@ -158,20 +163,58 @@ class ClockSampler:
 
 # ----------------------------------------------------------------- workload
 def decode_bytes(case, w) -> int:
-    """Algorithmic bytes of one attn_decode call: valid K and V, q, o (bf16), lse, lengths (+ page table)."""
-    kvb = int(case.seqlens_k.sum()) * w.Hkv * w.d * 2 * 2
+    """Algorithmic bytes of one attn_decode call: valid K and V (2 bytes per element,
+    1 for an FP8 cache, plus its scales), q, o (bf16), lse, lengths (+ page table)."""
+    eb = 1 if w.fp8 else 2
+    kvb = int(case.seqlens_k.sum()) * w.Hkv * w.d * eb * 2
+    scales = 2 * w.Hkv * 4 if w.fp8 else 0
     qo = 2 * w.B * w.T * w.Hq * w.d * 2
     lse = w.B * w.Hq * w.T * 4
     lens = w.B * 4
     table = 0
     if case.paged:
         table = int(sum((int(L) + 15) // 16 for L in case.seqlens_k)) * 4
-    return kvb + qo + lse + lens + table
+    return kvb + scales + qo + lse + lens + table
+
+
+def decode_flops(case, w) -> int:
+    """4 d FLOPs per visible (query row, key) pair; new token t of T sees keys
+    j <= L - T + t (causal) or all L keys."""
+    pairs = 0
+    for L in case.seqlens_k:
+        L = int(L)
+        pairs += w.T * (L - w.T) + w.T * (w.T + 1) // 2 if w.causal else w.T * L
+    return 4 * w.d * w.Hq * pairs
 
 
 def prefill_flops(w) -> int:
     pairs = w.N * (w.N + 1) // 2 if w.causal else w.N * w.N
     return 4 * w.B * w.Hq * w.d * pairs
+
+
+def append_and_attend(kv, wd, kc, vc, q, k_new, v_new, cache_lens, seqlens, table, scales, o, lse, msk, ws, stream,
+                      ev=None):
+    """kv_append then attn_decode (their FP8 forms for an FP8 cache); events 2 and 3 around the attend."""
+    if scales is None:
+        kv.kv_append(kc, vc, k_new, v_new, cache_lens, page_table=table, stream=stream)
+    else:
+        kv.kv_append_fp8(kc, vc, k_new, v_new, scales[0], scales[1], cache_lens, page_table=table, stream=stream)
+    if ev is not None:
+        ev[2].record(stream)
+    if scales is None:
+        kv.attn_decode(q, kc, vc, seqlens, o, lse, page_table=table, max_seqlen_k=msk, scale=wd.scale,
+                       causal=wd.causal, workspace=ws, stream=stream)
+    else:
+        kv.attn_decode_fp8(q, kc, vc, scales[0], scales[1], seqlens, o, lse, page_table=table, max_seqlen_k=msk,
+                           scale=wd.scale, causal=wd.causal, workspace=ws, stream=stream)
+    if ev is not None:
+        ev[3].record(stream)
+
+
+def decode_kernel_name(wd) -> str:
+    R = wd.Hq // wd.Hkv * wd.T
+    split = "decode_split_kernel" + ("<fp8>" if wd.fp8 else "") if R <= 32 else "decode_tc_kernel"
+    return f"{split} + decode_combine_kernel"
 
 
 def run_ours(args, world, rank, local):
@@ -191,7 +234,7 @@ def run_ours(args, world, rank, local):
     o = torch.empty(wp.B, wp.N, wp.Hq, wp.d, dtype=torch.bfloat16, device=dev)
     lse = torch.empty(wp.B, wp.Hq, wp.N, dtype=torch.float32, device=dev)
     case = synth.decode_inputs(wd.B, wd.T, wd.Hq, wd.Hkv, wd.d, wd.len_lo, wd.len_hi,
-                               synth.SEEDS[dec_name] + seed_off, device=dev, paged=wd.paged)
+                               synth.SEEDS[dec_name] + seed_off, device=dev, paged=wd.paged, fp8=wd.fp8)
     cache_lens = torch.as_tensor(case.cache_lens.astype(np.int32), device=dev)
     seqlens = torch.as_tensor(case.seqlens_k.astype(np.int32), device=dev)
     table = None if case.page_table is None else torch.as_tensor(case.page_table, device=dev)
@@ -202,6 +245,8 @@ def run_ours(args, world, rank, local):
     ld = torch.empty(wd.B, wd.Hq, wd.T, dtype=torch.float32, device=dev)
     ws = kv.decode_workspace(wd.B, wd.T, wd.Hq, wd.Hkv, wd.d, msk, 0, dev)
     stream = torch.cuda.current_stream(dev)
+    scales = ((torch.as_tensor(case.k_scale, device=dev), torch.as_tensor(case.v_scale, device=dev))
+              if wd.fp8 else None)
 
     def step(ev=None):
         if ev is not None:
@@ -210,13 +255,10 @@ def run_ours(args, world, rank, local):
         if ev is not None:
             ev[1].record(stream)
         # the same token position is appended every step, so the cache length stays fixed
-        kv.kv_append(kc, vc, case.k_new, case.v_new, cache_lens, page_table=table, stream=stream)
-        if ev is not None:
-            ev[2].record(stream)
-        kv.attn_decode(case.q, kc, vc, seqlens, od, ld, page_table=table, max_seqlen_k=msk, scale=wd.scale,
-                       causal=wd.causal, workspace=ws, stream=stream)
-        if ev is not None:
-            ev[3].record(stream)
+        append_and_attend(kv, wd, kc, vc, case.q, case.k_new, case.v_new, cache_lens, seqlens, table, scales, od,
+                          ld, msk, ws, stream, ev)
+
+
 
     kv.attn_get_device_status(clear=True)
     for _ in range(args.warmup):
@@ -254,17 +296,20 @@ def run_ours(args, world, rank, local):
     K = args.steps
     flops = prefill_flops(wp)
     dbytes = decode_bytes(case, wd)
+    dflops = decode_flops(case, wd)
 
     # whole-job: units summed over ranks / slowest rank's time
     tot_flops, pf_max = reduce_over_ranks(flops * K, pf_ms, world, dev)
     tot_bytes, dec_max = reduce_over_ranks(dbytes * K, dec_ms, world, dev)
+    tot_dflops, _ = reduce_over_ranks(dflops * K, dec_ms, world, dev)
     _, total_max = reduce_over_ranks(0.0, total_ms, world, dev)
     pf_tflops = tot_flops / (pf_max * 1e-3) / 1e12
     dec_gbs = tot_bytes / (dec_max * 1e-3) / 1e9
+    dec_tflops = tot_dflops / (dec_max * 1e-3) / 1e12
 
     # -------- end to end through the public API with host buffers (pinned)
     e2e = None if args.no_e2e else run_e2e(kv, torch, dev, stream, wp, wd, q, k, v, case, table, msk, ws, args,
-                                           world)
+                                           world, scales)
 
     peaks, peak_src = load_peaks()
     pf_kernel_tflops = flops / (pf_ms / K * 1e-3) / 1e12          # per launch, this rank
@@ -276,10 +321,20 @@ def run_ours(args, world, rank, local):
                "peak_source": f"{peak_src} (bf16 burst)", "traffic": traffic.get("prefill"),
                "kernel": "prefill_kernel<128>", "flops_per_launch": flops,
                "launch_ms": round(pf_ms / K, 4)}
-    roof_dec = {"bound": "hbm", "achieved": round(dec_kernel_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(dec_kernel_gbs / peaks["hbm_gbs"], 4), "peak_source": f"{peak_src} (copy)",
-                "traffic": traffic.get("decode"), "kernel": "decode_split_kernel + decode_combine_kernel",
-                "bytes_per_launch": dbytes, "launch_ms": round(dec_ms / K, 4)}
+    # the decode call is HBM-bound unless its flops per byte pass the ridge (many new tokens: chunked prefill)
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    dec_kernel_tflops = dflops / (dec_ms / K * 1e-3) / 1e12
+    if dflops / dbytes > ridge:
+        roof_dec = {"bound": "tensor", "achieved": round(dec_kernel_tflops, 1), "peak": peaks["bf16_tflops"],
+                    "unit": "TFLOP/s", "frac": round(dec_kernel_tflops / peaks["bf16_tflops"], 4),
+                    "frac_of_sustained": round(dec_kernel_tflops / peaks["bf16_tflops_sustained"], 4),
+                    "peak_source": f"{peak_src} (bf16 burst)", "traffic": None, "kernel": decode_kernel_name(wd),
+                    "flops_per_launch": dflops, "bytes_per_launch": dbytes, "launch_ms": round(dec_ms / K, 4)}
+    else:
+        roof_dec = {"bound": "hbm", "achieved": round(dec_kernel_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(dec_kernel_gbs / peaks["hbm_gbs"], 4), "peak_source": f"{peak_src} (copy)",
+                    "traffic": traffic.get("decode") if not wd.fp8 and wd.T * wd.Hq // wd.Hkv <= 32 else None,
+                    "kernel": decode_kernel_name(wd), "bytes_per_launch": dbytes, "launch_ms": round(dec_ms / K, 4)}
 
     out = None
     if rank == 0:
@@ -294,13 +349,14 @@ def run_ours(args, world, rank, local):
                             "causal": wp.causal, "o_dtype": "bf16"},
                 "decode": {"name": dec_name, "B": wd.B, "T": wd.T, "Hq": wd.Hq, "Hkv": wd.Hkv, "d": wd.d,
                            "cache_len": [wd.len_lo, wd.len_hi], "paged": wd.paged, "append_before_attend": True,
-                           "kv_bytes_per_step": int(case.seqlens_k.sum()) * wd.Hkv * wd.d * 4},
+                           "kv_dtype": "e4m3 + fp32 scale per KV head" if wd.fp8 else "bf16",
+                           "kv_bytes_per_step": int(case.seqlens_k.sum()) * wd.Hkv * wd.d * (2 if wd.fp8 else 4)},
                 "l2": "no flush: every step reads inputs larger than the 126 MB L2",
                 "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                 "seed": synth.SEEDS[pf_name],
             },
-            "decode": {"value": round(dec_gbs, 1), "unit": "GB/s", "roofline": roof_dec,
-                       "append_ms_per_step": round(ap_ms / K, 4)},
+            "decode": {"value": round(dec_gbs, 1), "unit": "GB/s", "tflops": round(dec_tflops, 2),
+                       "roofline": roof_dec, "append_ms_per_step": round(ap_ms / K, 4)},
             "roofline": roof_pf,
             "cpu_baseline": cpu,
             "e2e": e2e,
@@ -313,7 +369,7 @@ def run_ours(args, world, rank, local):
     return out
 
 
-def run_e2e(kv, torch, dev, stream, wp, wd, q, k, v, case, table, msk, ws, args, world):
+def run_e2e(kv, torch, dev, stream, wp, wd, q, k, v, case, table, msk, ws, args, world, scales=None):
     """Same step through the public API, inputs copied from pinned host memory
     and results read back every step (the KV cache stays resident: it is state)."""
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
@@ -351,9 +407,7 @@ def run_e2e(kv, torch, dev, stream, wp, wd, q, k, v, case, table, msk, ws, args,
         dvn.copy_(hvn, non_blocking=True)
         dcl.copy_(hcl, non_blocking=True)
         dsl.copy_(hsl, non_blocking=True)
-        kv.kv_append(kc, vc, dkn, dvn, dcl, page_table=table, stream=stream)
-        kv.attn_decode(ddq, kc, vc, dsl, ddo, ddl, page_table=table, max_seqlen_k=msk, scale=wd.scale,
-                       causal=wd.causal, workspace=ws, stream=stream)
+        append_and_attend(kv, wd, kc, vc, ddq, dkn, dvn, dcl, dsl, table, scales, ddo, ddl, msk, ws, stream)
         hdo.copy_(ddo, non_blocking=True)
         hdl.copy_(ddl, non_blocking=True)
         if ev is not None:
@@ -456,7 +510,7 @@ def oracle_decode_sample(wd, case_h, budget_s, rng):
         t0 = time.perf_counter()
         oracle.decode(qs, kc, vc, [L], wd.scale, wd.causal)
         t += time.perf_counter() - t0
-        nbytes += L * wd.d * 4 + 2 * wd.T * G * wd.d * 2
+        nbytes += L * wd.d * (2 if wd.fp8 else 4) + 2 * wd.T * G * wd.d * 2
         units += 1
         if t >= budget_s:
             return nbytes, t, units
@@ -464,8 +518,24 @@ def oracle_decode_sample(wd, case_h, budget_s, rng):
 
 def host_decode_case(case, wd, max_seqs=4):
     """fp64 host copies of a few sequences of the decode workload (cache as it is
-    after the append: stored rows followed by the new tokens)."""
+    after the append: stored rows followed by the new tokens; an FP8 cache is
+    dequantised, and its new tokens quantised, by the oracle)."""
     import torch
+
+    def values(rows, which):
+        if not wd.fp8:
+            return rows.float().cpu().numpy()
+        import oracle
+        s = case.k_scale if which == 0 else case.v_scale
+        return oracle.fp8.dequantize(rows.cpu().numpy(), s)
+
+    def new_values(rows, which):
+        if not wd.fp8:
+            return rows.float().cpu().numpy()
+        import oracle
+        s = case.k_scale if which == 0 else case.v_scale
+        return oracle.fp8.dequantize(oracle.fp8.quantize_rows(rows.float().cpu().numpy(), s), s)
+
     idx = list(range(min(max_seqs, wd.B)))
     Lmax = int(max(case.seqlens_k[i] for i in idx))
     k = np.zeros((len(idx), Lmax, wd.Hkv, wd.d))
@@ -479,10 +549,10 @@ def host_decode_case(case, wd, max_seqs=4):
             vb = case.v_pool.index_select(0, ids).reshape(nb * 16, wd.Hkv, wd.d)[:L0]
         else:
             kb, vb = case.k_cache[b, :L0], case.v_cache[b, :L0]
-        k[j, :L0] = kb.float().cpu().numpy()
-        v[j, :L0] = vb.float().cpu().numpy()
-        k[j, L0:L0 + wd.T] = case.k_new[b].float().cpu().numpy()
-        v[j, L0:L0 + wd.T] = case.v_new[b].float().cpu().numpy()
+        k[j, :L0] = values(kb, 0)
+        v[j, :L0] = values(vb, 1)
+        k[j, L0:L0 + wd.T] = new_values(case.k_new[b], 0)
+        v[j, L0:L0 + wd.T] = new_values(case.v_new[b], 1)
     return {"q": case.q[idx].float().cpu().numpy().astype(np.float64), "k": k, "v": v,
             "seqlens_k": case.seqlens_k[idx]}
 
@@ -508,7 +578,7 @@ def run_reference(args):
     q, k, v = synth.prefill_inputs(wp.B, wp.Hq, wp.Hkv, wp.N, wp.d, synth.SEEDS[pf_name], "cpu")
     n_seq = 2   # sequences of the decode workload held on the host for sampling
     case = synth.decode_inputs(n_seq, wd.T, wd.Hq, wd.Hkv, wd.d, wd.len_lo, wd.len_hi, synth.SEEDS[dec_name],
-                               device="cpu", paged=wd.paged)
+                               device="cpu", paged=wd.paged, fp8=wd.fp8)
     ch = host_decode_case(case, _shrink(wd, n_seq), max_seqs=n_seq)
     rng = np.random.default_rng(1)
     # each step is a bounded sample, sized so the whole run stays within a few minutes

@@ -69,7 +69,8 @@ enum {
   ATTN_DEV_PAGE_ID = 1,      /* a page-table entry read was outside [0, num_blocks) */
   ATTN_DEV_SEQLEN = 2,       /* seqlens_k[b] < T, > max_seqlen_k or beyond the cache capacity */
   ATTN_DEV_APPEND_RANGE = 4, /* kv_append position beyond the cache capacity / page table */
-  ATTN_DEV_TIMEOUT = 8       /* a bounded wait inside a kernel gave up (no fault, results invalid) */
+  ATTN_DEV_TIMEOUT = 8,      /* a bounded wait inside a kernel gave up (no fault, results invalid) */
+  ATTN_DEV_SCALE = 16        /* an FP8 cache scale was not a positive finite number */
 };
 
 /*
@@ -129,8 +130,12 @@ ATTN_API size_t attn_decode_workspace_bytes(int B, int T, int Hq, int Hkv, int d
  *               into at most n chunks
  *   workspace   device memory of at least attn_decode_workspace_bytes(...) bytes,
  *               16-byte aligned; contents on entry do not matter
- * Rows per KV head R = (Hq / Hkv) * T must be <= 128: R <= 32 runs on warp-level
- * MMAs, 33 <= R <= 128 on the tcgen05 tensor cores with the scores in TMEM.
+ * T may be large: a prompt chunk appended to a cached prefix (chunked prefill,
+ * prefix caching; [P1] "用它" enable-prefix-caching) is this same call with T =
+ * the chunk length, and T = seqlens_k[b] is a prefill from scratch.  With
+ * R = (Hq / Hkv) * T query rows per KV head, R <= 32 runs on warp-level MMAs;
+ * larger R on the tcgen05 tensor cores, in row tiles of whole tokens of at most
+ * 128 rows, scores in TMEM.  Hq / Hkv must be <= 128.
  * Errors: ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED (d, rows per KV head),
  * ATTN_ERR_WORKSPACE, ATTN_ERR_CUDA.  Bad lengths or page ids found on the
  * device set ATTN_DEV_SEQLEN / ATTN_DEV_PAGE_ID and make the affected rows NaN.
@@ -161,6 +166,51 @@ ATTN_API int attn_decode(const void* q, const void* k_cache, const void* v_cache
 ATTN_API int kv_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new, const int32_t* cache_lens,
               const int32_t* page_table, int max_blocks_per_seq, int num_blocks, int cache_capacity, int B, int T,
               int Hkv, int d, void* stream);
+
+/*
+ * attn_decode_fp8 -- attn_decode over an FP8 KV cache.
+ *
+ * Defines: [P1] "用它" (serving with an 8-bit float KV cache, --kv-cache-dtype
+ * fp8) and [P3] FlashAttention-3 paragraph of "背景" (FP8 mode combines
+ * quantisation with the tiled kernel); the attention itself is attn_decode's.
+ * The pages fix no encoding; this library stores OCP E4M3 ("FN") codes: one
+ * byte per element, exponent bias 7, largest finite +-448, no infinities.
+ * Cached element (token, head g, i) stands for value(code) * k_scale[g] (K) or
+ * value(code) * v_scale[g] (V); the result is exact attention over those values.
+ *
+ *   k_cache, v_cache  uint8 e4m3 codes in attn_decode's layouts (contiguous
+ *                     [B, cache_capacity, Hkv, d] or paged pools
+ *                     [num_blocks, 16, Hkv, d]): half the bytes of the bf16 cache
+ *   k_scale, v_scale  device fp32 [Hkv]; positive and finite, else the affected
+ *                     rows are NaN and ATTN_DEV_SCALE is set
+ *   everything else   as for attn_decode, including the workspace size
+ *                     (attn_decode_workspace_bytes with the same arguments)
+ * Built for d = 128 and at most 32 query rows per KV head ((Hq / Hkv) * T);
+ * other shapes return ATTN_ERR_UNSUPPORTED.  The products run on f16 tensor
+ * cores: every e4m3 value is exact in f16, q is rounded to f16 (exact for bf16
+ * values of magnitude 2^-14 .. 65504; larger magnitudes overflow) and the
+ * softmax weights are rounded to f16 before the P V product.
+ */
+ATTN_API int attn_decode_fp8(const void* q, const void* k_cache, const void* v_cache, const float* k_scale,
+                             const float* v_scale, const int32_t* seqlens_k, const int32_t* page_table,
+                             int max_blocks_per_seq, int num_blocks, int cache_capacity, int max_seqlen_k, void* o,
+                             int o_dtype, float* lse, int B, int T, int Hq, int Hkv, int d, float scale, int causal,
+                             int num_splits, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * kv_append_fp8 -- kv_append into an FP8 cache: quantise, then write.
+ *
+ * Each new value x (bf16) of KV head g is stored as the e4m3 code nearest to
+ * x / scale[g] (the quotient computed in fp32 by one IEEE division; ties to the
+ * even code; magnitudes beyond 448, infinities included, saturate to +-448;
+ * NaN stays NaN).  Placement, arguments and errors are kv_append's; k_scale
+ * and v_scale are device fp32 [Hkv] (positive and finite, else nothing is
+ * written for that head and ATTN_DEV_SCALE is set).  d must be 64 or 128.
+ */
+ATTN_API int kv_append_fp8(void* k_cache, void* v_cache, const void* k_new, const void* v_new, const float* k_scale,
+                           const float* v_scale, const int32_t* cache_lens, const int32_t* page_table,
+                           int max_blocks_per_seq, int num_blocks, int cache_capacity, int B, int T, int Hkv, int d,
+                           void* stream);
 
 /*
  * kv_cache_bytes -- bytes held by a KV cache: 2 * n_layers * batch * tokens *

@@ -21,11 +21,12 @@ import torch
 __all__ = [
     "lib", "LIB_PATH", "AttnError",
     "attn_prefill", "attn_decode", "attn_decode_workspace_bytes", "attn_decode_noalloc", "kv_append",
+    "attn_decode_fp8", "kv_append_fp8",
     "kv_cache_bytes", "ATTN_DECODE_NOALLOC_SCRATCH_BYTES",
     "attn_get_device_status", "attn_status_string", "decode_workspace",
     "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_WORKSPACE", "ATTN_ERR_CUDA",
     "ATTN_ERR_DEVICE", "ATTN_F32", "ATTN_BF16", "ATTN_DEV_PAGE_ID", "ATTN_DEV_SEQLEN",
-    "ATTN_DEV_APPEND_RANGE", "ATTN_DEV_TIMEOUT",
+    "ATTN_DEV_APPEND_RANGE", "ATTN_DEV_TIMEOUT", "ATTN_DEV_SCALE",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvattn.so")
@@ -33,7 +34,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvattn.s
 ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_WORKSPACE, ATTN_ERR_CUDA, ATTN_ERR_DEVICE = 0, -1, -2, -3, -4, -5
 ATTN_F32, ATTN_BF16 = 0, 1
 ATTN_DECODE_NOALLOC_SCRATCH_BYTES = 32 << 20
-ATTN_DEV_PAGE_ID, ATTN_DEV_SEQLEN, ATTN_DEV_APPEND_RANGE, ATTN_DEV_TIMEOUT = 1, 2, 4, 8
+ATTN_DEV_PAGE_ID, ATTN_DEV_SEQLEN, ATTN_DEV_APPEND_RANGE, ATTN_DEV_TIMEOUT, ATTN_DEV_SCALE = 1, 2, 4, 8, 16
 
 _p, _i, _i64, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
 
@@ -44,7 +45,10 @@ _SIGNATURES = {
                          _p]),
     "attn_decode_noalloc": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _p, _i, _p, _i, _i, _i, _i, _i, _f, _i, _i,
                                  _p]),
+    "attn_decode_fp8": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _p, _i, _p, _i, _i, _i, _i, _i, _f, _i,
+                             _i, _p, _sz, _p]),
     "kv_append": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p]),
+    "kv_append_fp8": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p]),
     "kv_cache_bytes": (_i64, [_i, _i, _i64, _i, _i, _i]),
     "attn_get_device_status": (_i, [_i]),
     "attn_status_string": (ctypes.c_char_p, [_i]),
@@ -195,6 +199,62 @@ def kv_append(k_cache, v_cache, k_new, v_new, cache_lens, page_table=None, strea
                        None if page_table is None else _dev(page_table, "page_table", torch.int32),
                        max_blocks, num_blocks, cap, B, T, Hkv, d, _stream(stream))
     _check("kv_append", st)
+
+
+_CODES = (torch.uint8, torch.float8_e4m3fn)
+
+
+def _codes(t: torch.Tensor, name: str) -> int:
+    """An FP8 cache: e4m3 codes held as uint8 or torch.float8_e4m3fn."""
+    if t.dtype not in _CODES:
+        raise ValueError(f"{name} must hold e4m3 codes (uint8 or float8_e4m3fn)")
+    return _dev(t, name)
+
+
+def attn_decode_fp8(q, k_cache, v_cache, k_scale, v_scale, seqlens_k, o, lse=None, page_table=None, max_seqlen_k=0,
+                    scale=None, causal=True, num_splits=0, workspace=None, stream=None) -> None:
+    """``attn_decode`` over an FP8 cache: k/v hold e4m3 codes (uint8 or float8_e4m3fn,
+    same shapes as the bf16 cache); k_scale/v_scale float32 ``[Hkv]``."""
+    B, T, Hq, d = q.shape
+    max_blocks, num_blocks, cap, Hkv = _cache_geometry(k_cache, page_table)
+    if tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(o.shape) != (B, T, Hq, d):
+        raise ValueError("shape mismatch")
+    if tuple(k_scale.shape) != (Hkv,) or tuple(v_scale.shape) != (Hkv,):
+        raise ValueError("k_scale and v_scale must be [Hkv]")
+    if lse is not None and tuple(lse.shape) != (B, Hq, T):
+        raise ValueError("lse must be [B, Hq, T]")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if workspace is None:
+        msk = max_seqlen_k if max_seqlen_k else (cap if page_table is None else max_blocks * 16)
+        workspace = decode_workspace(B, T, Hq, Hkv, d, msk, num_splits, q.device)
+    st = lib.attn_decode_fp8(_dev(q, "q", torch.bfloat16), _codes(k_cache, "k_cache"), _codes(v_cache, "v_cache"),
+                             _dev(k_scale, "k_scale", torch.float32), _dev(v_scale, "v_scale", torch.float32),
+                             _dev(seqlens_k, "seqlens_k", torch.int32),
+                             None if page_table is None else _dev(page_table, "page_table", torch.int32),
+                             max_blocks, num_blocks, cap, int(max_seqlen_k), _dev(o, "o"), _out_dtype(o),
+                             None if lse is None else _dev(lse, "lse", torch.float32), B, T, Hq, Hkv, d, scale,
+                             int(bool(causal)), int(num_splits), _dev(workspace, "workspace"),
+                             workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("attn_decode_fp8", st)
+
+
+def kv_append_fp8(k_cache, v_cache, k_new, v_new, k_scale, v_scale, cache_lens, page_table=None,
+                  stream=None) -> None:
+    """Quantise bf16 k_new/v_new ``[B, T, Hkv, d]`` with the per-KV-head scales and
+    write the e4m3 codes at positions cache_lens[b] + t."""
+    B, T, Hkv, d = k_new.shape
+    max_blocks, num_blocks, cap, Hkv_c = _cache_geometry(k_cache, page_table)
+    if Hkv_c != Hkv or tuple(v_new.shape) != tuple(k_new.shape) or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("shape mismatch")
+    if tuple(k_scale.shape) != (Hkv,) or tuple(v_scale.shape) != (Hkv,):
+        raise ValueError("k_scale and v_scale must be [Hkv]")
+    st = lib.kv_append_fp8(_codes(k_cache, "k_cache"), _codes(v_cache, "v_cache"),
+                           _dev(k_new, "k_new", torch.bfloat16), _dev(v_new, "v_new", torch.bfloat16),
+                           _dev(k_scale, "k_scale", torch.float32), _dev(v_scale, "v_scale", torch.float32),
+                           _dev(cache_lens, "cache_lens", torch.int32),
+                           None if page_table is None else _dev(page_table, "page_table", torch.int32),
+                           max_blocks, num_blocks, cap, B, T, Hkv, d, _stream(stream))
+    _check("kv_append_fp8", st)
 
 
 def kv_cache_bytes(n_layers, batch, tokens, n_kv_heads, head_dim, elem_bytes) -> int:

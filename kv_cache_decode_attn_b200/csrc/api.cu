@@ -53,22 +53,24 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 }  // namespace
 
 int encode_tmap_nd(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
-                   const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+                   const cuuint64_t* strides_bytes, const cuuint32_t* box, int elem_bytes) {
   auto fn = get_encode_fn();
-  if (!fn || rank < 1 || rank > 5) return 1;
+  if (!fn || rank < 1 || rank > 5 || (elem_bytes != 1 && elem_bytes != 2)) return 1;
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims,
+  const CUtensorMapDataType dt = elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUresult r = fn(map, dt, (cuuint32_t)rank, const_cast<void*>(base), dims,
                   strides_bytes, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? 0 : 1;
 }
 
 int encode_tmap_3d(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2,
-                   uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1, uint32_t box2) {
+                   uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1, uint32_t box2,
+                   int elem_bytes) {
   cuuint64_t dims[3] = {dim0, dim1, dim2};
   cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
   cuuint32_t box[3] = {box0, box1, box2};
-  return encode_tmap_nd(map, base, 3, dims, strides, box);
+  return encode_tmap_nd(map, base, 3, dims, strides, box, elem_bytes);
 }
 
 }  // namespace kvattn
@@ -87,7 +89,7 @@ bool decode_layout(int B, int T, int Hq, int Hkv, int d, int max_seqlen_k, int n
   if (d != 64 && d != 128) return false;
   DecodeLayout L;
   L.R = (Hq / Hkv) * T;
-  L.chunk = decode_chunk_tokens(B, Hkv, L.R, max_seqlen_k, num_splits);
+  L.chunk = decode_chunk_tokens(B, T, Hq / Hkv, Hkv, max_seqlen_k, num_splits);
   L.max_chunks = (max_seqlen_k + L.chunk - 1) / L.chunk;
   const size_t items = (size_t)B * Hkv * L.max_chunks;
   L.o_bytes = items * L.R * d * sizeof(float);
@@ -180,11 +182,17 @@ int attn_prefill(const void* q, const void* k, const void* v, void* o, int o_dty
   return cuda_status(launch_prefill(a, static_cast<cudaStream_t>(stream)), "attn_prefill");
 }
 
-int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens_k,
-                const int32_t* page_table, int max_blocks_per_seq, int num_blocks, int cache_capacity,
-                int max_seqlen_k, void* o, int o_dtype, float* lse, int B, int T, int Hq, int Hkv, int d,
-                float scale, int causal, int num_splits, void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+int decode_impl(const void* q, const void* k_cache, const void* v_cache, const float* k_scale, const float* v_scale,
+                bool fp8, const int32_t* seqlens_k, const int32_t* page_table, int max_blocks_per_seq,
+                int num_blocks, int cache_capacity, int max_seqlen_k, void* o, int o_dtype, float* lse, int B, int T,
+                int Hq, int Hkv, int d, float scale, int causal, int num_splits, void* workspace,
+                size_t workspace_bytes, void* stream, const char* name) {
   if (!q || !k_cache || !v_cache || !seqlens_k || !o) return ATTN_ERR_INVALID_ARG;
+  if (fp8 && (!k_scale || !v_scale)) return ATTN_ERR_INVALID_ARG;
   if (B < 1 || T < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || num_splits < 0) return ATTN_ERR_INVALID_ARG;
   if (o_dtype != ATTN_F32 && o_dtype != ATTN_BF16) return ATTN_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale) || (causal != 0 && causal != 1)) return ATTN_ERR_INVALID_ARG;
@@ -202,7 +210,9 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
   if (max_seqlen_k == 0) max_seqlen_k = capacity_tokens;
   if (max_seqlen_k < T || max_seqlen_k > capacity_tokens) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-  if ((Hq / Hkv) * T > 128) return ATTN_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 128) return ATTN_ERR_UNSUPPORTED;                       // one token's heads must fit a row tile
+  if (fp8 && (Hq / Hkv) * T > kDecodeMmaRows) return ATTN_ERR_UNSUPPORTED;
+  if (fp8 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
   DecodeLayout L;
   if (!decode_layout(B, T, Hq, Hkv, d, max_seqlen_k, num_splits, &L)) return ATTN_ERR_INVALID_ARG;
@@ -234,13 +244,18 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
   a.part_o = static_cast<float*>(workspace);
   a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + L.lse_offset);
   a.status = st;
-  return cuda_status(launch_decode(a, static_cast<cudaStream_t>(stream)), "attn_decode");
+  a.fp8 = fp8 ? 1 : 0;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
+  return cuda_status(launch_decode(a, static_cast<cudaStream_t>(stream)), name);
 }
 
-int kv_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new, const int32_t* cache_lens,
-              const int32_t* page_table, int max_blocks_per_seq, int num_blocks, int cache_capacity, int B, int T,
-              int Hkv, int d, void* stream) {
+int append_impl(void* k_cache, void* v_cache, const void* k_new, const void* v_new, const float* k_scale,
+                const float* v_scale, bool fp8, const int32_t* cache_lens, const int32_t* page_table,
+                int max_blocks_per_seq, int num_blocks, int cache_capacity, int B, int T, int Hkv, int d, void* stream,
+                const char* name) {
   if (!k_cache || !v_cache || !k_new || !v_new || !cache_lens) return ATTN_ERR_INVALID_ARG;
+  if (fp8 && (!k_scale || !v_scale)) return ATTN_ERR_INVALID_ARG;
   if (B < 1 || T < 1 || Hkv < 1) return ATTN_ERR_INVALID_ARG;
   if (page_table) {
     if (max_blocks_per_seq < 1 || num_blocks < 1) return ATTN_ERR_INVALID_ARG;
@@ -267,7 +282,47 @@ int kv_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new
   a.Hkv = Hkv;
   a.d = d;
   a.status = st;
-  return cuda_status(launch_append(a, static_cast<cudaStream_t>(stream)), "kv_append");
+  a.fp8 = fp8 ? 1 : 0;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
+  return cuda_status(launch_append(a, static_cast<cudaStream_t>(stream)), name);
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens_k,
+                const int32_t* page_table, int max_blocks_per_seq, int num_blocks, int cache_capacity,
+                int max_seqlen_k, void* o, int o_dtype, float* lse, int B, int T, int Hq, int Hkv, int d,
+                float scale, int causal, int num_splits, void* workspace, size_t workspace_bytes, void* stream) {
+  return decode_impl(q, k_cache, v_cache, nullptr, nullptr, false, seqlens_k, page_table, max_blocks_per_seq,
+                     num_blocks, cache_capacity, max_seqlen_k, o, o_dtype, lse, B, T, Hq, Hkv, d, scale, causal,
+                     num_splits, workspace, workspace_bytes, stream, "attn_decode");
+}
+
+int attn_decode_fp8(const void* q, const void* k_cache, const void* v_cache, const float* k_scale,
+                    const float* v_scale, const int32_t* seqlens_k, const int32_t* page_table, int max_blocks_per_seq,
+                    int num_blocks, int cache_capacity, int max_seqlen_k, void* o, int o_dtype, float* lse, int B,
+                    int T, int Hq, int Hkv, int d, float scale, int causal, int num_splits, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  return decode_impl(q, k_cache, v_cache, k_scale, v_scale, true, seqlens_k, page_table, max_blocks_per_seq,
+                     num_blocks, cache_capacity, max_seqlen_k, o, o_dtype, lse, B, T, Hq, Hkv, d, scale, causal,
+                     num_splits, workspace, workspace_bytes, stream, "attn_decode_fp8");
+}
+
+int kv_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new, const int32_t* cache_lens,
+              const int32_t* page_table, int max_blocks_per_seq, int num_blocks, int cache_capacity, int B, int T,
+              int Hkv, int d, void* stream) {
+  return append_impl(k_cache, v_cache, k_new, v_new, nullptr, nullptr, false, cache_lens, page_table,
+                     max_blocks_per_seq, num_blocks, cache_capacity, B, T, Hkv, d, stream, "kv_append");
+}
+
+int kv_append_fp8(void* k_cache, void* v_cache, const void* k_new, const void* v_new, const float* k_scale,
+                  const float* v_scale, const int32_t* cache_lens, const int32_t* page_table, int max_blocks_per_seq,
+                  int num_blocks, int cache_capacity, int B, int T, int Hkv, int d, void* stream) {
+  return append_impl(k_cache, v_cache, k_new, v_new, k_scale, v_scale, true, cache_lens, page_table,
+                     max_blocks_per_seq, num_blocks, cache_capacity, B, T, Hkv, d, stream, "kv_append_fp8");
 }
 
 }  // extern "C"

@@ -12,11 +12,23 @@
 // chunk's normalised output and log-sum-exp go to the workspace; a second
 // kernel merges the chunks of each row with the log-sum-exp combine.
 //
+// FP8 caches (e4m3 codes with one float32 scale per KV head for K and for V):
+// the tile is half as many bytes; each consumer thread reads its K and V bytes
+// with 16-byte shared loads and converts them exactly to f16 with the hardware
+// e4m3x2 -> f16x2 conversion, so the MMAs run in f16 (Q and P are rounded to
+// f16).  The sum over d in Q K^T may take the d positions in any order as long
+// as Q uses the same order, so a thread's four consecutive K bytes of a row
+// feed one k16 step directly; for P V the output columns are permuted the same
+// way (column n of the j-th 8-column block is d = 16 n + j) so that a thread's
+// V bytes of two keys pair up with one byte permute.  The K scale is folded
+// into the softmax scale and the V scale into the chunk's normalisation.
+//
 // Method: "[BEE-30062] FlashAttention 與高效注意力核心", sections "背景" and
 // "為長上下文推論啟用 FlashDecoding" (split along the KV length, numerically
 // stable reduction of partial softmax results); "大模型面試笔记——Attention篇"
 // section 2 (online safe softmax); "Effizienz", "Der wichtige Maskenfehler beim
-// Cache" (bottom-right aligned mask for several new tokens).
+// Cache" (bottom-right aligned mask for several new tokens); "KV cache, flash
+// attention and inference optimisation" lesson, section "用它" (an FP8 KV cache).
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -29,15 +41,17 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-template <int D, int MT>
+template <int D, int MT, bool FP8>
 struct DecodeCfg {
+  static_assert(!FP8 || D == 128, "FP8 caches are built for d = 128");
   static constexpr int kConsumerWarps = 4 * MT;
   static constexpr int kThreads = 32 * (kConsumerWarps + 1);
-  static constexpr int kHalves = D / 64;              // 128-byte swizzle spans 64 bf16
+  static constexpr int kHalves = (FP8 ? D : 2 * D) / 128;   // 128-byte swizzle spans per token row
   static constexpr int kHalfBytes = kDecodeTile * 128;
   static constexpr int kTensorBytes = kHalves * kHalfBytes;   // one of K or V per stage
   static constexpr int kStageBytes = 2 * kTensorBytes;
-  static constexpr int kStages = (MT == 1) ? (D == 128 ? 3 : 6) : (D == 128 ? 4 : 8);
+  static constexpr int kBf16Stages = (MT == 1) ? (D == 128 ? 3 : 6) : (D == 128 ? 4 : 8);
+  static constexpr int kStages = FP8 ? 2 * kBf16Stages : kBf16Stages;   // the same bytes in flight
   static constexpr int kRedStride = D + 8;            // floats per row of the merge buffer
   static constexpr int kRedBytes = MT * 4 * 16 * kRedStride * 4;
   static_assert(kRedBytes <= kStages * kStageBytes, "merge buffer must fit in the ring");
@@ -49,6 +63,8 @@ struct DecodeCfg {
 
 struct SplitParams {
   const __nv_bfloat16* q;
+  const float* k_scale;   // FP8 caches: per-KV-head scales (else unused)
+  const float* v_scale;
   const int32_t* seqlens;
   const int32_t* page_table;
   float* part_o;
@@ -67,11 +83,16 @@ __device__ __forceinline__ bool seqlen_bad(int L, int T, int max_seqlen, bool pa
   return false;
 }
 
-template <int D, int MT, bool PAGED>
-__global__ void __launch_bounds__(DecodeCfg<D, MT>::kThreads, DecodeCfg<D, MT>::kMinBlocks)
+// bf16 pair (low = lower index) -> f16 pair
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
+  return pack_f16x2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+}
+
+template <int D, int MT, bool PAGED, bool FP8>
+__global__ void __launch_bounds__(DecodeCfg<D, MT, FP8>::kThreads, DecodeCfg<D, MT, FP8>::kMinBlocks)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const SplitParams p) {
-  using C = DecodeCfg<D, MT>;
+  using C = DecodeCfg<D, MT, FP8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
@@ -92,6 +113,18 @@ __global__ void __launch_bounds__(DecodeCfg<D, MT>::kThreads, DecodeCfg<D, MT>::
   if (tok_begin >= L) return;
   const int tok_end = min(tok_begin + p.chunk, L);
   const int n_tiles = (tok_end - tok_begin + kDecodeTile - 1) / kDecodeTile;
+  float scale_log2 = p.scale_log2, v_scale = 1.f;
+  if constexpr (FP8) {
+    const float ks = __ldg(p.k_scale + g), vs = __ldg(p.v_scale + g);
+    if (!(ks > 0.f && ks <= 3.402823466e38f && vs > 0.f && vs <= 3.402823466e38f)) {
+      if (threadIdx.x == 0 && c == 0) atomicOr(p.status, DEV_SCALE);
+      const size_t item = ((size_t)b * p.Hkv + g) * p.max_chunks + c;
+      for (int r = threadIdx.x; r < p.R; r += blockDim.x) p.part_lse[item * p.R + r] = NAN;
+      return;   // the whole CTA leaves before any barrier: the scales are uniform across it
+    }
+    scale_log2 *= ks;
+    v_scale = vs;
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -181,13 +214,28 @@ __global__ void __launch_bounds__(DecodeCfg<D, MT>::kThreads, DecodeCfg<D, MT>::
     };
     const __nv_bfloat16* qr0 = r0 < p.R ? qrow(r0) : nullptr;
     const __nv_bfloat16* qr1 = r1 < p.R ? qrow(r1) : nullptr;
+    if constexpr (!FP8) {
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const int c0 = kk * 16 + tig * 2;
-      qa[kk][0] = qr0 ? *reinterpret_cast<const uint32_t*>(qr0 + c0) : 0u;
-      qa[kk][1] = qr1 ? *reinterpret_cast<const uint32_t*>(qr1 + c0) : 0u;
-      qa[kk][2] = qr0 ? *reinterpret_cast<const uint32_t*>(qr0 + c0 + 8) : 0u;
-      qa[kk][3] = qr1 ? *reinterpret_cast<const uint32_t*>(qr1 + c0 + 8) : 0u;
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const int c0 = kk * 16 + tig * 2;
+        qa[kk][0] = qr0 ? *reinterpret_cast<const uint32_t*>(qr0 + c0) : 0u;
+        qa[kk][1] = qr1 ? *reinterpret_cast<const uint32_t*>(qr1 + c0) : 0u;
+        qa[kk][2] = qr0 ? *reinterpret_cast<const uint32_t*>(qr0 + c0 + 8) : 0u;
+        qa[kk][3] = qr1 ? *reinterpret_cast<const uint32_t*>(qr1 + c0 + 8) : 0u;
+      }
+    } else {
+      // k16 step kk takes d = 16 (tig + 4 (kk / 4)) + 4 (kk % 4) + {0, 1 | 2, 3}: the
+      // four consecutive K bytes this thread reads for that step
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const int d0 = 16 * (tig + 4 * (kk >> 2)) + 4 * (kk & 3);
+        const uint2 x0 = qr0 ? *reinterpret_cast<const uint2*>(qr0 + d0) : make_uint2(0u, 0u);
+        const uint2 x1 = qr1 ? *reinterpret_cast<const uint2*>(qr1 + d0) : make_uint2(0u, 0u);
+        qa[kk][0] = bf16x2_to_f16x2(x0.x);
+        qa[kk][1] = bf16x2_to_f16x2(x1.x);
+        qa[kk][2] = bf16x2_to_f16x2(x0.y);
+        qa[kk][3] = bf16x2_to_f16x2(x1.y);
+      }
     }
   }
 
@@ -216,7 +264,7 @@ __global__ void __launch_bounds__(DecodeCfg<D, MT>::kThreads, DecodeCfg<D, MT>::
     float sacc[2][4];
 #pragma unroll
     for (int n = 0; n < 2; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
-    {
+    if constexpr (!FP8) {
       const int trow = wsub * 16 + (lm >> 1) * 8 + lr;   // token row inside the tile
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
@@ -228,13 +276,51 @@ __global__ void __launch_bounds__(DecodeCfg<D, MT>::kThreads, DecodeCfg<D, MT>::
         mma_bf16_16816(sacc[0], qa[kk], b0, b1);
         mma_bf16_16816(sacc[1], qa[kk], b2, b3);
       }
+    } else {
+      // token rows gid (n8 block 0) and 8 + gid (block 1); 16-byte chunks tig and tig + 4
+      uint32_t kw[2][8];
+#pragma unroll
+      for (int nb = 0; nb < 2; ++nb) {
+        const int trow = wsub * 16 + nb * 8 + gid;       // trow & 7 == gid
+        const uint32_t ra = kbase + trow * 128;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const uint4 x = lds128(ra + (((tig + 4 * hh) ^ gid) << 4));
+          kw[nb][4 * hh + 0] = x.x;
+          kw[nb][4 * hh + 1] = x.y;
+          kw[nb][4 * hh + 2] = x.z;
+          kw[nb][4 * hh + 3] = x.w;
+        }
+      }
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb) {
+          const uint32_t w = kw[nb][kk];
+          mma_f16_16816(sacc[nb], qa[kk], e4m3x2_to_f16x2(w), e4m3x2_to_f16x2(w >> 16));
+        }
+      }
     }
 
     // ---- V fragments for this warp's 16 tokens, loaded before the softmax so the
     //      shared-memory latency overlaps it; keys at or past L may hold anything
     //      (even NaN), so their V rows are zeroed
-    uint32_t vb[D / 16][4];
-    {
+    uint32_t vb[FP8 ? 1 : D / 16][4];
+    uint32_t vw[FP8 ? 4 : 1][4];   // FP8: 16 bytes (d = 16 gid .. 16 gid + 15) of keys 2tig, 2tig+1, 2tig+8, 2tig+9
+    if constexpr (FP8) {
+      const bool tail = tok_base + 16 > L;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int key = 2 * tig + (i & 1) + 8 * (i >> 1);
+        const int vrow = wsub * 16 + key;
+        uint4 x = lds128(vbase + vrow * 128 + ((gid ^ (vrow & 7)) << 4));
+        if (tail && tok_base + key >= L) x = make_uint4(0u, 0u, 0u, 0u);
+        vw[i][0] = x.x;
+        vw[i][1] = x.y;
+        vw[i][2] = x.z;
+        vw[i][3] = x.w;
+      }
+    } else {
       const bool tail = tok_base + 16 > L;
       const int vrow = wsub * 16 + (lm & 1) * 8 + lr;
       const int ta = tok_base + tig * 2, tb = ta + 8;
@@ -266,7 +352,7 @@ __global__ void __launch_bounds__(DecodeCfg<D, MT>::kThreads, DecodeCfg<D, MT>::
       for (int e = 0; e < 4; ++e) {
         const int tok = tok_base + n * 8 + tig * 2 + (e & 1);
         const int end = (e < 2) ? end0 : end1;
-        const float v = (tok < end) ? sacc[n][e] * p.scale_log2 : -INFINITY;
+        const float v = (tok < end) ? sacc[n][e] * scale_log2 : -INFINITY;
         sacc[n][e] = v;
         if (e < 2) mx0 = fmaxf(mx0, v); else mx1 = fmaxf(mx1, v);
       }
@@ -306,16 +392,35 @@ __global__ void __launch_bounds__(DecodeCfg<D, MT>::kThreads, DecodeCfg<D, MT>::
     l0 += ps0;
     l1 += ps1;
     uint32_t pa[4];
-    pa[0] = pack_bf16x2(sacc[0][0], sacc[0][1]);
-    pa[1] = pack_bf16x2(sacc[0][2], sacc[0][3]);
-    pa[2] = pack_bf16x2(sacc[1][0], sacc[1][1]);
-    pa[3] = pack_bf16x2(sacc[1][2], sacc[1][3]);
+    if constexpr (!FP8) {
+      pa[0] = pack_bf16x2(sacc[0][0], sacc[0][1]);
+      pa[1] = pack_bf16x2(sacc[0][2], sacc[0][3]);
+      pa[2] = pack_bf16x2(sacc[1][0], sacc[1][1]);
+      pa[3] = pack_bf16x2(sacc[1][2], sacc[1][3]);
 
-    // ---- O += P V
+      // ---- O += P V
 #pragma unroll
-    for (int nn = 0; nn < D / 16; ++nn) {
-      mma_bf16_16816(o_acc[2 * nn], pa, vb[nn][0], vb[nn][1]);
-      mma_bf16_16816(o_acc[2 * nn + 1], pa, vb[nn][2], vb[nn][3]);
+      for (int nn = 0; nn < D / 16; ++nn) {
+        mma_bf16_16816(o_acc[2 * nn], pa, vb[nn][0], vb[nn][1]);
+        mma_bf16_16816(o_acc[2 * nn + 1], pa, vb[nn][2], vb[nn][3]);
+      }
+    } else {
+      pa[0] = pack_f16x2(sacc[0][0], sacc[0][1]);
+      pa[1] = pack_f16x2(sacc[0][2], sacc[0][3]);
+      pa[2] = pack_f16x2(sacc[1][0], sacc[1][1]);
+      pa[3] = pack_f16x2(sacc[1][2], sacc[1][3]);
+      // ---- O += P V over 16 blocks of 8 output columns; block j, column n is d = 16 n + j,
+      //      i.e. byte j of this thread's 16 V bytes; a byte permute pairs keys (2tig, 2tig+1)
+      //      and (2tig+8, 2tig+9) for blocks j and j + 1
+#pragma unroll
+      for (int jj = 0; jj < D / 16; ++jj) {
+        const int w = jj >> 1;
+        const uint32_t sel = (jj & 1) ? 0x7362u : 0x5140u;
+        const uint32_t x01 = prmt(vw[0][w], vw[1][w], sel);
+        const uint32_t x23 = prmt(vw[2][w], vw[3][w], sel);
+        mma_f16_16816(o_acc[2 * jj], pa, e4m3x2_to_f16x2(x01), e4m3x2_to_f16x2(x23));
+        mma_f16_16816(o_acc[2 * jj + 1], pa, e4m3x2_to_f16x2(x01 >> 16), e4m3x2_to_f16x2(x23 >> 16));
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
@@ -354,10 +459,18 @@ __global__ void __launch_bounds__(DecodeCfg<D, MT>::kThreads, DecodeCfg<D, MT>::
   float* red = reinterpret_cast<float*>(smem) + ((mt * 4 + wsub) * 16) * C::kRedStride;
 #pragma unroll
   for (int n = 0; n < D / 8; ++n) {
-    const int col = n * 8 + tig * 2;
-    *reinterpret_cast<float2*>(red + gid * C::kRedStride + col) = make_float2(o_acc[n][0] * f0, o_acc[n][1] * f0);
-    *reinterpret_cast<float2*>(red + (gid + 8) * C::kRedStride + col) =
-        make_float2(o_acc[n][2] * f1, o_acc[n][3] * f1);
+    if constexpr (!FP8) {
+      const int col = n * 8 + tig * 2;
+      *reinterpret_cast<float2*>(red + gid * C::kRedStride + col) = make_float2(o_acc[n][0] * f0, o_acc[n][1] * f0);
+      *reinterpret_cast<float2*>(red + (gid + 8) * C::kRedStride + col) =
+          make_float2(o_acc[n][2] * f1, o_acc[n][3] * f1);
+    } else {
+      const int col = 32 * tig + n;   // columns 2tig and 2tig + 1 of block n are d = 32 tig + n and + 16
+      red[gid * C::kRedStride + col] = o_acc[n][0] * f0;
+      red[gid * C::kRedStride + col + 16] = o_acc[n][1] * f0;
+      red[(gid + 8) * C::kRedStride + col] = o_acc[n][2] * f1;
+      red[(gid + 8) * C::kRedStride + col + 16] = o_acc[n][3] * f1;
+    }
   }
   asm volatile("bar.sync 1, %0;" ::"n"(C::kConsumerWarps * 32) : "memory");
 
@@ -384,7 +497,7 @@ __global__ void __launch_bounds__(DecodeCfg<D, MT>::kThreads, DecodeCfg<D, MT>::
       acc.z += x.z;
       acc.w += x.w;
     }
-    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+    const float inv = lsum > 0.f ? (FP8 ? v_scale / lsum : 1.f / lsum) : 0.f;
     *reinterpret_cast<float4*>(out + (size_t)r * D + col) =
         make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
     if (col == 0) p.part_lse[item * p.R + r] = lsum > 0.f ? (mrow + log2f(lsum)) * kLn2 : -INFINITY;
@@ -492,11 +605,11 @@ __global__ void __launch_bounds__(256, 4) decode_combine_kernel(const float* __r
   if (lse && lane == 0) lse[((size_t)b * p.Hq + h) * p.T + t] = lse_row;
 }
 
-template <int D, int MT, bool PAGED>
+template <int D, int MT, bool PAGED, bool FP8 = false>
 cudaError_t run_split(const CUtensorMap& tk, const CUtensorMap& tv, const SplitParams& sp, int B,
                       cudaStream_t stream) {
-  using C = DecodeCfg<D, MT>;
-  auto kern = decode_split_kernel<D, MT, PAGED>;
+  using C = DecodeCfg<D, MT, FP8>;
+  auto kern = decode_split_kernel<D, MT, PAGED, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(sp.max_chunks, sp.Hkv, B);
@@ -506,7 +619,7 @@ cudaError_t run_split(const CUtensorMap& tk, const CUtensorMap& tv, const SplitP
 
 }  // namespace
 
-int decode_chunk_tokens(int B, int Hkv, int rows, int max_seqlen, int num_splits) {
+int decode_chunk_tokens(int B, int T, int G, int Hkv, int max_seqlen, int num_splits) {
   int chunk;
   if (num_splits > 0) {
     chunk = (max_seqlen + num_splits - 1) / num_splits;
@@ -514,9 +627,11 @@ int decode_chunk_tokens(int B, int Hkv, int rows, int max_seqlen, int num_splits
     // Long chunks stream longer and leave fewer partials to merge; measured on
     // B200 the best were 2048 tokens for 16 x 8 sequence-heads up to 32K keys and
     // 4096 for 8 x 8 up to 128K.  Start at 4096 and halve until the grid holds
-    // about 14 work items per SM (counted as if every sequence had max_seqlen).
+    // about 14 work items per SM (counted as if every sequence had max_seqlen;
+    // row tiles of many new tokens count as separate items).
+    const long long units = (long long)B * Hkv * decode_row_tiles(T, G);
     chunk = 4096;
-    while (chunk > 256 && (long long)B * Hkv * ((max_seqlen + chunk - 1) / chunk) < 2048) chunk >>= 1;
+    while (chunk > 256 && units * ((max_seqlen + chunk - 1) / chunk) < 2048) chunk >>= 1;
   }
   // a multiple of both kernels' tiles
   chunk = ((chunk + kDecodeTcTile - 1) / kDecodeTcTile) * kDecodeTcTile;
@@ -528,6 +643,8 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
   const int G = a.Hq / a.Hkv, R = G * a.T;
   SplitParams sp;
   sp.q = static_cast<const __nv_bfloat16*>(a.q);
+  sp.k_scale = a.k_scale;
+  sp.v_scale = a.v_scale;
   sp.seqlens = a.seqlens;
   sp.page_table = a.page_table;
   sp.part_o = a.part_o;
@@ -552,13 +669,21 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
   const bool tc = R > kDecodeMmaRows;
   const uint32_t box_rows = paged ? kPageTokens : (tc ? kDecodeTcTile : kDecodeTile);
   CUtensorMap tk, tv;
-  const uint64_t s1 = (uint64_t)a.d * 2, s2 = (uint64_t)a.Hkv * a.d * 2;
-  if (encode_tmap_3d(&tk, a.k, a.d, a.Hkv, rows, s1, s2, 64, 1, box_rows) ||
-      encode_tmap_3d(&tv, a.v, a.d, a.Hkv, rows, s1, s2, 64, 1, box_rows))
+  const int eb = a.fp8 ? 1 : 2;   // bytes per cached element
+  const uint64_t s1 = (uint64_t)a.d * eb, s2 = (uint64_t)a.Hkv * a.d * eb;
+  const uint32_t box0 = 128 / eb;  // one 128-byte swizzle span
+  if (encode_tmap_3d(&tk, a.k, a.d, a.Hkv, rows, s1, s2, box0, 1, box_rows, eb) ||
+      encode_tmap_3d(&tv, a.v, a.d, a.Hkv, rows, s1, s2, box0, 1, box_rows, eb))
     return cudaErrorInvalidValue;
 
   cudaError_t e;
-  if (tc) {
+  if (a.fp8) {
+    // api.cu admits d == 128 and at most kDecodeMmaRows rows per KV head
+    if (R <= 16) e = paged ? run_split<128, 1, true, true>(tk, tv, sp, a.B, stream)
+                           : run_split<128, 1, false, true>(tk, tv, sp, a.B, stream);
+    else e = paged ? run_split<128, 2, true, true>(tk, tv, sp, a.B, stream)
+                   : run_split<128, 2, false, true>(tk, tv, sp, a.B, stream);
+  } else if (tc) {
     e = launch_decode_tc(a, tk, tv, stream);
   } else if (a.d == 128) {
     if (R <= 16) e = paged ? run_split<128, 1, true>(tk, tv, sp, a.B, stream) : run_split<128, 1, false>(tk, tv, sp, a.B, stream);

@@ -1,12 +1,15 @@
-// Split-KV decode attention on the sm_100a tensor cores, for many query rows per
-// KV head (R = (Hq/Hkv) * T from 33 to 128: grouped heads times several new
-// tokens, e.g. a speculative-verify step of 8 or 16 tokens).
+// Split-KV attention of T new tokens against a KV cache on the sm_100a tensor
+// cores, for many query rows per KV head (R = (Hq/Hkv) * T above 32: grouped
+// heads times several new tokens -- a speculative-verify step of 8 or 16
+// tokens, or a whole prompt chunk appended to an existing cache, which is
+// chunked prefill / prefill against a cached prefix).
 //
-// One CTA owns one work item (key chunk c, KV head g, sequence b), exactly like
-// the warp-MMA decode kernel, and writes the same per-chunk partials (normalised
-// O and log-sum-exp per row) that the combine kernel merges.  The R query rows
-// of KV head g form one 128-row tcgen05 tile (row r = t * G + hh; rows >= R are
-// zero).  Warp roles:
+// The rows of KV head g are numbered r = t * G + hh (token t, grouped head hh)
+// and cut into row tiles of TT whole tokens (TT * G <= 128 rows, the tcgen05 M).
+// One CTA owns one work item (row tile, key chunk c, KV head g, sequence b) and
+// writes the same per-chunk partials (normalised O and log-sum-exp per row) that
+// the combine kernel merges.  With the bottom-right mask a row tile only reads
+// keys up to the last one its last token sees.  Warp roles:
 //   warps 0..3  softmax: thread i owns row i (TMEM lane i); warps whose rows are
 //               all >= R stay idle;
 //   warp 4      TMA producer: Q once, then 128-token K/V tiles (contiguous: one
@@ -69,7 +72,8 @@ struct TcParams {
   float* part_o;
   float* part_lse;
   unsigned* status;
-  int T, Hq, Hkv, G, R;
+  int T, Hq, Hkv, G, R;   // R = G * T rows per KV head (the partials' row count)
+  int TT;                 // tokens per row tile (TT * G <= 128)
   int chunk, max_chunks, capacity, max_blocks, num_blocks, max_seqlen;
   float scale_log2;
   int causal;
@@ -96,17 +100,29 @@ __global__ void __launch_bounds__(192, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int c = blockIdx.x % p.max_chunks, rt = blockIdx.x / p.max_chunks, g = blockIdx.y, b = blockIdx.z;
   const int L = p.seqlens[b];
   // invalid lengths are reported (and their rows made NaN) by the combine kernel
   if (L < p.T || L > p.max_seqlen || (!PAGED && L > p.capacity) ||
       (PAGED && (L + kPageTokens - 1) / kPageTokens > p.max_blocks))
     return;
   const int tok_begin = c * p.chunk;
-  if (tok_begin >= L) return;
-  const int tok_end = min(tok_begin + p.chunk, L);
+  if (tok_begin >= L) return;   // the combine reads only chunks that start before L
+  const int t0 = rt * p.TT;                      // first token of this row tile
+  const int tile_tokens = min(p.TT, p.T - t0);
+  const int tile_rows = tile_tokens * p.G;       // live rows: 0 .. tile_rows - 1
+  const size_t item = ((size_t)b * p.Hkv + g) * p.max_chunks + c;
+  const size_t row0 = item * p.R + (size_t)t0 * p.G;   // partial row of tile row 0
+  int tok_end = min(tok_begin + p.chunk, L);
+  if (p.causal) tok_end = min(tok_end, L - p.T + t0 + tile_tokens);   // last token's first invisible key
+  if (tok_end <= tok_begin) {
+    // no key of this chunk is visible to any row of the tile: an empty partial
+    for (int i = threadIdx.x; i < tile_rows * D; i += blockDim.x) p.part_o[row0 * D + i] = 0.f;
+    for (int r = threadIdx.x; r < tile_rows; r += blockDim.x) p.part_lse[row0 + r] = -INFINITY;
+    return;
+  }
   const int n_tiles = (tok_end - tok_begin + kTok - 1) / kTok;
-  const int active_warps = (p.R + 31) / 32;
+  const int active_warps = (tile_rows + 31) / 32;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[T_Q], 1);
@@ -124,12 +140,14 @@ __global__ void __launch_bounds__(192, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  // rows R..127 of the Q tile are never loaded: make them zero (whole 128-byte rows)
+  // rows TT*G..127 of the Q tile are never loaded: make them zero (whole 128-byte rows);
+  // rows of tokens >= T inside the box are zero-filled by the copy
   {
-    const int per_half = (kRows - p.R) * 8;   // 16-byte chunks of rows R..127 in one half of d
+    const int box_rows = p.TT * p.G;
+    const int per_half = (kRows - box_rows) * 8;   // 16-byte chunks of rows box_rows..127 in one half of d
     for (int i = threadIdx.x; i < per_half * C::kHalves; i += blockDim.x) {
       const int half = i / per_half, rem = i - half * per_half;
-      *reinterpret_cast<uint4*>(smem + C::kQOff + half * C::kHalfBytes + p.R * 128 + rem * 16) =
+      *reinterpret_cast<uint4*>(smem + C::kQOff + half * C::kHalfBytes + box_rows * 128 + rem * 16) =
           make_uint4(0, 0, 0, 0);
     }
   }
@@ -149,11 +167,12 @@ __global__ void __launch_bounds__(192, 1)
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       const uint64_t pol = policy_evict_first();
-      // Q rows (t, head g*G + hh) for t < T, hh < G: one box {64, G, T, 1} per half of d
-      mbar_arrive_expect_tx(&bars[T_Q], p.R * D * 2);
+      // Q rows (t, head g*G + hh) for t0 <= t < t0 + TT, hh < G: one box {64, G, TT, 1} per half
+      // of d (the full box is counted, also where tokens >= T are zero-filled)
+      mbar_arrive_expect_tx(&bars[T_Q], p.TT * p.G * D * 2);
 #pragma unroll
       for (int hh = 0; hh < C::kHalves; ++hh)
-        tma_load_4d(smem + C::kQOff + hh * C::kHalfBytes, &tmQ, &bars[T_Q], hh * 64, g * p.G, 0, b, pol);
+        tma_load_4d(smem + C::kQOff + hh * C::kHalfBytes, &tmQ, &bars[T_Q], hh * 64, g * p.G, t0, b, pol);
       int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};
       constexpr int kBlocks = kTok / kPageTokens;
       // physical blocks of one tile, read together (the copies' memory clobbers
@@ -261,9 +280,9 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp < active_warps) {
     // ------------------------------------------------------------- softmax warps
     const int row = warp * 32 + lane;
-    const bool live = row < p.R;
+    const bool live = row < tile_rows;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    const int t = live ? row / p.G : 0;
+    const int t = live ? t0 + row / p.G : 0;
     const int end = p.causal ? L - p.T + t + 1 : L;       // first invisible key of this row
     float m = -INFINITY, l = 0.f;
     bool ok = true;
@@ -334,9 +353,11 @@ __global__ void __launch_bounds__(192, 1)
           tmem_st32(lane_base + C::kOCol + cc, r);
         }
       }
-      // keys at or past L may hold anything (even NaN): zero their V rows, which
-      // the PV MMA would otherwise multiply by p = 0
-      const int valid = L - key0;
+      // keys at or past this CTA's end may hold anything (past L: any bytes; past a
+      // row tile's last visible key in a paged cache: blocks never loaded, stale
+      // shared memory), even NaN: zero their V rows, which the PV MMA would
+      // otherwise multiply by p = 0
+      const int valid = tok_end - key0;
       if (valid < kTok && warp == 0) {
         if (!tc_wait(&bars[T_VFULL + st], (i >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
         uint8_t* vst = smem + C::kVOff + st * C::kTileBytes;
@@ -355,8 +376,7 @@ __global__ void __launch_bounds__(192, 1)
     // ---------------------------------------------------------- epilogue
     if (ok && tc_wait(&bars[T_OFINAL], 0, abort_flag, p.status) && !*abort_flag) {
       tc_fence_after();
-      const size_t item = ((size_t)b * p.Hkv + g) * p.max_chunks + c;
-      float* out = p.part_o + (item * p.R + row) * D;
+      float* out = p.part_o + (row0 + row) * D;
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
       for (int cc = 0; cc < D; cc += 32) {
@@ -371,9 +391,9 @@ __global__ void __launch_bounds__(192, 1)
                             __uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
         }
       }
-      if (live) p.part_lse[item * p.R + row] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+      if (live) p.part_lse[row0 + row] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
     } else if (live) {
-      p.part_lse[(((size_t)b * p.Hkv + g) * p.max_chunks + c) * p.R + row] = NAN;   // a wait gave up
+      p.part_lse[row0 + row] = NAN;   // a wait gave up
     }
   }
 
@@ -394,11 +414,13 @@ template <int D, bool PAGED>
 cudaError_t run_tc(const DecodeLaunch& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream) {
   using C = TcCfg<D>;
   const int G = a.Hq / a.Hkv;
+  const int TT = decode_tc_tile_tokens(a.T, G);
+  const int row_tiles = (a.T + TT - 1) / TT;
   CUtensorMap tq;
-  // q [B, T, Hq, d] as {d, Hq, T, B}; one box covers the G heads of a KV head for every new token
+  // q [B, T, Hq, d] as {d, Hq, T, B}; one box covers the G heads of a KV head for TT tokens
   cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)a.Hq, (cuuint64_t)a.T, (cuuint64_t)a.B};
   cuuint64_t str[3] = {(cuuint64_t)D * 2, (cuuint64_t)a.Hq * D * 2, (cuuint64_t)a.T * a.Hq * D * 2};
-  cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)a.T, 1};
+  cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)TT, 1};
   if (encode_tmap_nd(&tq, a.q, 4, dims, str, box)) return cudaErrorInvalidValue;
   TcParams p;
   p.seqlens = a.seqlens;
@@ -411,6 +433,7 @@ cudaError_t run_tc(const DecodeLaunch& a, const CUtensorMap& tk, const CUtensorM
   p.Hkv = a.Hkv;
   p.G = G;
   p.R = G * a.T;
+  p.TT = TT;
   p.chunk = a.chunk;
   p.max_chunks = a.max_chunks;
   p.capacity = a.capacity;
@@ -422,7 +445,8 @@ cudaError_t run_tc(const DecodeLaunch& a, const CUtensorMap& tk, const CUtensorM
   auto kern = decode_tc_kernel<D, PAGED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.max_chunks, a.Hkv, a.B);
+  if ((long long)a.max_chunks * row_tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
+  dim3 grid(a.max_chunks * row_tiles, a.Hkv, a.B);
   kern<<<grid, 192, C::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }

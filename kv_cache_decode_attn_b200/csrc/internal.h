@@ -34,6 +34,9 @@ struct DecodeLaunch {
   float* part_o;      // [B, Hkv, max_chunks, R, d]
   float* part_lse;    // [B, Hkv, max_chunks, R]
   unsigned* status;
+  int fp8 = 0;                    // k/v hold e4m3 codes with per-KV-head scales
+  const float* k_scale = nullptr;  // [Hkv]
+  const float* v_scale = nullptr;
 };
 
 struct PrefillLaunch {
@@ -59,20 +62,35 @@ struct AppendLaunch {
   int max_blocks, num_blocks, capacity;
   int B, T, Hkv, d;
   unsigned* status;
+  int fp8 = 0;                    // quantise the new rows to e4m3 with per-KV-head scales
+  const float* k_scale = nullptr;
+  const float* v_scale = nullptr;
 };
 
 // Tokens per split for attn_decode (host heuristic, deterministic in its inputs).
-int decode_chunk_tokens(int B, int Hkv, int rows, int max_seqlen, int num_splits);
+int decode_chunk_tokens(int B, int T, int G, int Hkv, int max_seqlen, int num_splits);
 
-// Encode a rank-N (1..5) bf16 tiled tensor map with 128-byte swizzle; strides
-// in bytes for dims 1..N-1.  Returns 0 on success.
+// Tokens per row tile of the tensor-core decode kernel (G query heads per KV head):
+// as many whole tokens as fit in 128 rows, at most T.
+inline int decode_tc_tile_tokens(int T, int G) { return T < 128 / G ? T : 128 / G; }
+// Row tiles per KV head: 1 on the warp-MMA path (at most kDecodeMmaRows rows).
+inline int decode_row_tiles(int T, int G) {
+  if (G * T <= kDecodeMmaRows) return 1;
+  const int tt = decode_tc_tile_tokens(T, G);
+  return (T + tt - 1) / tt;
+}
+
+// Encode a rank-N (1..5) tiled tensor map with 128-byte swizzle over bf16
+// (elem_bytes 2) or bytes (elem_bytes 1); strides in bytes for dims 1..N-1.
+// Returns 0 on success.
 int encode_tmap_nd(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
-                   const cuuint64_t* strides_bytes, const cuuint32_t* box);
+                   const cuuint64_t* strides_bytes, const cuuint32_t* box, int elem_bytes = 2);
 
-// Encode a 3-D bf16 tiled tensor map {inner, mid, rows} with 128-byte swizzle.
+// Encode a 3-D tiled tensor map {inner, mid, rows} with 128-byte swizzle.
 // Strides are in bytes for dims 1 and 2.  Returns 0 on success.
 int encode_tmap_3d(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2,
-                   uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1, uint32_t box2);
+                   uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1, uint32_t box2,
+                   int elem_bytes = 2);
 
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream);
 // tcgen05 split kernel for more than 16 query rows per KV head (K/V maps with 128-row boxes when contiguous)

@@ -1,11 +1,13 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers with bounded waits, TMA tile
-// loads, warp-level bf16 MMA, ldmatrix, ex2, and the tcgen05 / TMEM family.
+// loads, warp-level bf16/f16 MMA, ldmatrix, e4m3 conversions, ex2, and the
+// tcgen05 / TMEM family.
 // Every wait here is bounded: after the limit it reports failure to the caller,
 // which records a device status bit and leaves its loop; nothing traps.
 #pragma once
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace kvattn {
@@ -16,6 +18,7 @@ enum : unsigned {
   DEV_SEQLEN = 2u,
   DEV_APPEND_RANGE = 4u,
   DEV_TIMEOUT = 8u,
+  DEV_SCALE = 16u,
 };
 
 // wall-clock limit of one bounded wait, in nanoseconds (%globaltimer)
@@ -145,6 +148,50 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       "{%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// D (16x8 f32) += A (16x16 f16, row) * B (16x8 f16, col)
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Two e4m3 codes (low byte -> low half) to two f16 values; exact, every e4m3
+// value is an f16 value.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+  uint32_t d;
+  const unsigned short a = (unsigned short)(two_codes & 0xffffu);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"(a));
+  return d;
+}
+
+// Two f32 values to two e4m3 codes (lo -> low byte), round to nearest even,
+// saturating to +-448 (NaN stays NaN).
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+  unsigned short d;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// byte permute: result byte i = byte sel_i of the 8-byte value {b, a} (a = bytes 0..3)
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -86,6 +86,10 @@ WORKLOADS = {
                                 len_hi=32768, fp8=True),
     "decode_paged_fp8": Decode("decode_paged_fp8", B=8, T=1, Hq=64, Hkv=8, d=128, len_lo=32768,
                                len_hi=131072, paged=True, fp8=True),
+    # prefill against an existing cache: a 512-token prompt chunk appended to a
+    # cached prefix of 4K..16K tokens (chunked prefill / prefix caching)
+    "prefill_chunk_paged": Decode("prefill_chunk_paged", B=4, T=512, Hq=32, Hkv=8, d=128, len_lo=4096,
+                                  len_hi=16384, paged=True),
 }
 
 SEEDS = {name: 1000 + i for i, name in enumerate(WORKLOADS)}

@@ -94,7 +94,7 @@ def test_decode_rejects_bad_arguments():
     assert call(T=4, msk=3) == kv.ATTN_ERR_INVALID_ARG        # fewer keys than new tokens
     assert call(pt=P, mb=0, nb=10) == kv.ATTN_ERR_INVALID_ARG
     assert call(d=80) == kv.ATTN_ERR_UNSUPPORTED
-    assert call(Hq=64, Hkv=1, T=4) == kv.ATTN_ERR_UNSUPPORTED   # 256 rows per KV head
+    assert call(Hq=256, Hkv=1) == kv.ATTN_ERR_UNSUPPORTED       # 256 query heads per KV head > one row tile
     assert call(ws=None) == kv.ATTN_ERR_WORKSPACE
     assert call(wsb=16) == kv.ATTN_ERR_WORKSPACE
     assert call(ns=-1) == kv.ATTN_ERR_INVALID_ARG
@@ -108,6 +108,43 @@ def test_append_rejects_bad_arguments():
     assert L.kv_append(P, P, P, P, P, None, 0, 0, 0, 1, 1, 2, 128, None) == kv.ATTN_ERR_INVALID_ARG
     assert L.kv_append(P, P, P, P, P, P, 0, 5, 0, 1, 1, 2, 128, None) == kv.ATTN_ERR_INVALID_ARG
     assert L.kv_append(P, P, P, P, P, None, 0, 0, 10, 1, 1, 2, 72, None) == kv.ATTN_ERR_UNSUPPORTED
+
+
+def test_decode_fp8_rejects_bad_arguments():
+    L = kv.lib
+
+    def call(**kw):
+        a = dict(q=P, k=P, v=P, ks=P, vs=P, sl=P, pt=None, mb=0, nb=0, cap=100, msk=0, o=P, od=0, lse=None, B=2, T=1,
+                 Hq=8, Hkv=2, d=128, scale=0.1, causal=1, ns=0, ws=P, wsb=1 << 30)
+        a.update(kw)
+        return L.attn_decode_fp8(a["q"], a["k"], a["v"], a["ks"], a["vs"], a["sl"], a["pt"], a["mb"], a["nb"],
+                                 a["cap"], a["msk"], a["o"], a["od"], a["lse"], a["B"], a["T"], a["Hq"], a["Hkv"],
+                                 a["d"], a["scale"], a["causal"], a["ns"], a["ws"], a["wsb"], None)
+
+    assert call(ks=None) == kv.ATTN_ERR_INVALID_ARG
+    assert call(vs=None) == kv.ATTN_ERR_INVALID_ARG
+    assert call(q=None) == kv.ATTN_ERR_INVALID_ARG
+    assert call(d=64) == kv.ATTN_ERR_UNSUPPORTED               # FP8 decode is built for d = 128
+    assert call(Hq=36, Hkv=1) == kv.ATTN_ERR_UNSUPPORTED       # 36 rows per KV head > 32
+    assert call(Hq=8, Hkv=1, T=5) == kv.ATTN_ERR_UNSUPPORTED   # 40 rows
+    assert call(wsb=16) == kv.ATTN_ERR_WORKSPACE
+    assert call(T=4, msk=3) == kv.ATTN_ERR_INVALID_ARG
+
+
+def test_append_fp8_rejects_bad_arguments():
+    L = kv.lib
+    assert L.kv_append_fp8(P, P, P, P, None, P, P, None, 0, 0, 10, 1, 1, 2, 128, None) == kv.ATTN_ERR_INVALID_ARG
+    assert L.kv_append_fp8(P, P, P, P, P, None, P, None, 0, 0, 10, 1, 1, 2, 128, None) == kv.ATTN_ERR_INVALID_ARG
+    assert L.kv_append_fp8(P, P, P, P, P, P, None, None, 0, 0, 10, 1, 1, 2, 128, None) == kv.ATTN_ERR_INVALID_ARG
+    assert L.kv_append_fp8(P, P, P, P, P, P, P, None, 0, 0, 10, 1, 1, 2, 96, None) == kv.ATTN_ERR_UNSUPPORTED
+
+
+def test_binding_checks_fp8_cache_dtype():
+    import torch
+    x = torch.zeros(1, 4, 2, 128, dtype=torch.bfloat16)
+    s = torch.ones(2)
+    with pytest.raises(ValueError):
+        kv.attn_decode_fp8(x, x, x, s, s, torch.zeros(1, dtype=torch.int32), torch.zeros(1, 4, 2, 128))
 
 
 def test_binding_refuses_host_tensors():
