@@ -49,9 +49,12 @@ WORKLOAD_SETS = {
     # the same layer with an FP8 (e4m3, per-KV-head scales) KV cache
     "llama8b_layer_fp8": ("prefill_llama8b", "decode_contig_fp8"),
     "llama8b_paged_fp8": ("prefill_llama8b", "decode_paged_fp8"),
-    # prefill against an existing cache: 512-token prompt chunks on cached 4K..16K prefixes
+    # prefill against an existing cache: 512-token prompt chunks on cached 4K..16K prefixes,
+    # through attn_prefill_cache (the prefill kernel) or attn_decode (split-KV, row-tiled)
+    "llama8b_prefill_cache": ("prefill_llama8b", "prefill_chunk_paged"),
     "llama8b_chunked_prefill": ("prefill_llama8b", "prefill_chunk_paged"),
 }
+PREFILL_CACHE_SETS = {"llama8b_prefill_cache"}   # sets whose attend step is attn_prefill_cache
 DEFAULT_SET = "llama8b_layer"
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -193,15 +196,19 @@ def prefill_flops(w) -> int:
 
 
 def append_and_attend(kv, wd, kc, vc, q, k_new, v_new, cache_lens, seqlens, table, scales, o, lse, msk, ws, stream,
-                      ev=None):
-    """kv_append then attn_decode (their FP8 forms for an FP8 cache); events 2 and 3 around the attend."""
+                      ev=None, prefill_cache=False):
+    """kv_append then attn_decode (their FP8 forms for an FP8 cache, or attn_prefill_cache);
+    events 2 and 3 around the attend."""
     if scales is None:
         kv.kv_append(kc, vc, k_new, v_new, cache_lens, page_table=table, stream=stream)
     else:
         kv.kv_append_fp8(kc, vc, k_new, v_new, scales[0], scales[1], cache_lens, page_table=table, stream=stream)
     if ev is not None:
         ev[2].record(stream)
-    if scales is None:
+    if prefill_cache:
+        kv.attn_prefill_cache(q, kc, vc, seqlens, o, lse, page_table=table, scale=wd.scale, causal=wd.causal,
+                              stream=stream)
+    elif scales is None:
         kv.attn_decode(q, kc, vc, seqlens, o, lse, page_table=table, max_seqlen_k=msk, scale=wd.scale,
                        causal=wd.causal, workspace=ws, stream=stream)
     else:
@@ -211,7 +218,9 @@ def append_and_attend(kv, wd, kc, vc, q, k_new, v_new, cache_lens, seqlens, tabl
         ev[3].record(stream)
 
 
-def decode_kernel_name(wd) -> str:
+def decode_kernel_name(wd, prefill_cache=False) -> str:
+    if prefill_cache:
+        return "prefill_kernel<128, paged cache>" if wd.paged else "prefill_kernel<128, cache>"
     R = wd.Hq // wd.Hkv * wd.T
     split = "decode_split_kernel" + ("<fp8>" if wd.fp8 else "") if R <= 32 else "decode_tc_kernel"
     return f"{split} + decode_combine_kernel"
@@ -247,6 +256,7 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.current_stream(dev)
     scales = ((torch.as_tensor(case.k_scale, device=dev), torch.as_tensor(case.v_scale, device=dev))
               if wd.fp8 else None)
+    prefill_cache = args.workload in PREFILL_CACHE_SETS
 
     def step(ev=None):
         if ev is not None:
@@ -256,7 +266,7 @@ def run_ours(args, world, rank, local):
             ev[1].record(stream)
         # the same token position is appended every step, so the cache length stays fixed
         append_and_attend(kv, wd, kc, vc, case.q, case.k_new, case.v_new, cache_lens, seqlens, table, scales, od,
-                          ld, msk, ws, stream, ev)
+                          ld, msk, ws, stream, ev, prefill_cache)
 
 
 
@@ -309,7 +319,7 @@ def run_ours(args, world, rank, local):
 
     # -------- end to end through the public API with host buffers (pinned)
     e2e = None if args.no_e2e else run_e2e(kv, torch, dev, stream, wp, wd, q, k, v, case, table, msk, ws, args,
-                                           world, scales)
+                                           world, scales, prefill_cache)
 
     peaks, peak_src = load_peaks()
     pf_kernel_tflops = flops / (pf_ms / K * 1e-3) / 1e12          # per launch, this rank
@@ -328,13 +338,15 @@ def run_ours(args, world, rank, local):
         roof_dec = {"bound": "tensor", "achieved": round(dec_kernel_tflops, 1), "peak": peaks["bf16_tflops"],
                     "unit": "TFLOP/s", "frac": round(dec_kernel_tflops / peaks["bf16_tflops"], 4),
                     "frac_of_sustained": round(dec_kernel_tflops / peaks["bf16_tflops_sustained"], 4),
-                    "peak_source": f"{peak_src} (bf16 burst)", "traffic": None, "kernel": decode_kernel_name(wd),
+                    "peak_source": f"{peak_src} (bf16 burst)", "traffic": None,
+                    "kernel": decode_kernel_name(wd, prefill_cache),
                     "flops_per_launch": dflops, "bytes_per_launch": dbytes, "launch_ms": round(dec_ms / K, 4)}
     else:
         roof_dec = {"bound": "hbm", "achieved": round(dec_kernel_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": round(dec_kernel_gbs / peaks["hbm_gbs"], 4), "peak_source": f"{peak_src} (copy)",
                     "traffic": traffic.get("decode") if not wd.fp8 and wd.T * wd.Hq // wd.Hkv <= 32 else None,
-                    "kernel": decode_kernel_name(wd), "bytes_per_launch": dbytes, "launch_ms": round(dec_ms / K, 4)}
+                    "kernel": decode_kernel_name(wd, prefill_cache), "bytes_per_launch": dbytes,
+                    "launch_ms": round(dec_ms / K, 4)}
 
     out = None
     if rank == 0:
@@ -360,7 +372,8 @@ def run_ours(args, world, rank, local):
             "roofline": roof_pf,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": 4 * K,   # prefill, append, decode split, decode combine per step
+            # per step: prefill, append, then decode split + combine (or one attn_prefill_cache launch)
+            "gpu_launches": (3 if prefill_cache else 4) * K,
             "clocks": clocks.summary(),
         }
     if world > 1:
@@ -369,7 +382,8 @@ def run_ours(args, world, rank, local):
     return out
 
 
-def run_e2e(kv, torch, dev, stream, wp, wd, q, k, v, case, table, msk, ws, args, world, scales=None):
+def run_e2e(kv, torch, dev, stream, wp, wd, q, k, v, case, table, msk, ws, args, world, scales=None,
+            prefill_cache=False):
     """Same step through the public API, inputs copied from pinned host memory
     and results read back every step (the KV cache stays resident: it is state)."""
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
@@ -407,7 +421,8 @@ def run_e2e(kv, torch, dev, stream, wp, wd, q, k, v, case, table, msk, ws, args,
         dvn.copy_(hvn, non_blocking=True)
         dcl.copy_(hcl, non_blocking=True)
         dsl.copy_(hsl, non_blocking=True)
-        append_and_attend(kv, wd, kc, vc, ddq, dkn, dvn, dcl, dsl, table, scales, ddo, ddl, msk, ws, stream)
+        append_and_attend(kv, wd, kc, vc, ddq, dkn, dvn, dcl, dsl, table, scales, ddo, ddl, msk, ws, stream,
+                          prefill_cache=prefill_cache)
         hdo.copy_(ddo, non_blocking=True)
         hdl.copy_(ddl, non_blocking=True)
         if ev is not None:

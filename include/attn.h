@@ -96,6 +96,35 @@ ATTN_API int attn_prefill(const void* q, const void* k, const void* v, void* o, 
                  int Hkv, int N, int d, float scale, int causal, void* stream);
 
 /*
+ * attn_prefill_cache -- prefill against an existing KV cache: Nq new query
+ * tokens per sequence (a prompt chunk, or a prompt after a cached prefix)
+ * attend to every cached key plus themselves.
+ *
+ * Defines: attn_prefill's computation with the keys read from the cache;
+ * [P5] "Der wichtige Maskenfehler beim Cache" (the Nq queries are the LAST Nq
+ * positions: with causal = 1, query i sees keys j <= seqlens_k[b] - Nq + i) and
+ * [P1] "用它" / exercise 2 of its "运动" (prefix caching: the prompt prefix's
+ * K,V are computed once and reused).  Same result as attn_decode with T = Nq,
+ * computed by the prefill kernel (no key split, no workspace): the faster
+ * choice for chunks of some hundred tokens or more.
+ *
+ *   q           device bf16 [B, Nq, Hq, d]
+ *   k_cache,    as for attn_decode (contiguous [B, cache_capacity, Hkv, d], or
+ *   v_cache     paged pools [num_blocks, 16, Hkv, d] with page_table)
+ *   seqlens_k   device int32 [B]: keys of sequence b INCLUDING the Nq new ones
+ *               (append them with kv_append first, on the same stream)
+ *   o, lse      [B, Nq, Hq, d] of o_dtype; fp32 [B, Hq, Nq] or NULL
+ * Errors: ATTN_ERR_INVALID_ARG (including a capacity below Nq),
+ * ATTN_ERR_UNSUPPORTED (d), ATTN_ERR_CUDA.  A length below Nq or beyond the
+ * capacity sets ATTN_DEV_SEQLEN and makes that sequence's rows NaN; bad page ids
+ * set ATTN_DEV_PAGE_ID.
+ */
+ATTN_API int attn_prefill_cache(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens_k,
+                                const int32_t* page_table, int max_blocks_per_seq, int num_blocks, int cache_capacity,
+                                void* o, int o_dtype, float* lse, int B, int Nq, int Hq, int Hkv, int d, float scale,
+                                int causal, void* stream);
+
+/*
  * attn_decode_workspace_bytes -- bytes of device workspace attn_decode needs
  * for these sizes (the per-chunk partial outputs and log-sum-exps of the split
  * along the keys).  num_splits as for attn_decode.  Returns 0 for invalid sizes.

@@ -21,7 +21,7 @@ import torch
 __all__ = [
     "lib", "LIB_PATH", "AttnError",
     "attn_prefill", "attn_decode", "attn_decode_workspace_bytes", "attn_decode_noalloc", "kv_append",
-    "attn_decode_fp8", "kv_append_fp8",
+    "attn_decode_fp8", "kv_append_fp8", "attn_prefill_cache",
     "kv_cache_bytes", "ATTN_DECODE_NOALLOC_SCRATCH_BYTES",
     "attn_get_device_status", "attn_status_string", "decode_workspace",
     "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_WORKSPACE", "ATTN_ERR_CUDA",
@@ -41,6 +41,7 @@ _p, _i, _i64, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_
 _SIGNATURES = {
     "attn_prefill": (_i, [_p, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _f, _i, _p]),
     "attn_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "attn_prefill_cache": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _p, _i, _p, _i, _i, _i, _i, _i, _f, _i, _p]),
     "attn_decode": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _p, _i, _p, _i, _i, _i, _i, _i, _f, _i, _i, _p, _sz,
                          _p]),
     "attn_decode_noalloc": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _p, _i, _p, _i, _i, _i, _i, _i, _f, _i, _i,
@@ -122,6 +123,27 @@ def attn_prefill(q, k, v, o, lse=None, scale=None, causal=True, stream=None) -> 
                           _dev(o, "o"), _out_dtype(o), None if lse is None else _dev(lse, "lse", torch.float32),
                           B, Hq, Hkv, N, d, scale, int(bool(causal)), _stream(stream))
     _check("attn_prefill", st)
+
+
+def attn_prefill_cache(q, k_cache, v_cache, seqlens_k, o, lse=None, page_table=None, scale=None, causal=True,
+                       stream=None) -> None:
+    """Prefill of q ``[B, Nq, Hq, d]`` against a cache (contiguous ``[B, cap, Hkv, d]`` or pools
+    ``[nblk, 16, Hkv, d]`` with page_table int32 ``[B, max_blocks]``) already holding the Nq new
+    tokens; seqlens_k int32 ``[B]`` counts them too.  o ``[B, Nq, Hq, d]``, lse ``[B, Hq, Nq]``."""
+    B, Nq, Hq, d = q.shape
+    max_blocks, num_blocks, cap, Hkv = _cache_geometry(k_cache, page_table)
+    if tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(o.shape) != (B, Nq, Hq, d):
+        raise ValueError("shape mismatch")
+    if lse is not None and tuple(lse.shape) != (B, Hq, Nq):
+        raise ValueError("lse must be [B, Hq, Nq]")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    st = lib.attn_prefill_cache(_dev(q, "q", torch.bfloat16), _dev(k_cache, "k_cache", torch.bfloat16),
+                                _dev(v_cache, "v_cache", torch.bfloat16), _dev(seqlens_k, "seqlens_k", torch.int32),
+                                None if page_table is None else _dev(page_table, "page_table", torch.int32),
+                                max_blocks, num_blocks, cap, _dev(o, "o"), _out_dtype(o),
+                                None if lse is None else _dev(lse, "lse", torch.float32), B, Nq, Hq, Hkv, d, scale,
+                                int(bool(causal)), _stream(stream))
+    _check("attn_prefill_cache", st)
 
 
 def attn_decode_workspace_bytes(B, T, Hq, Hkv, d, max_seqlen_k, num_splits=0) -> int:

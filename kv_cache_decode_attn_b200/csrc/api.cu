@@ -292,6 +292,50 @@ int append_impl(void* k_cache, void* v_cache, const void* k_new, const void* v_n
 
 extern "C" {
 
+int attn_prefill_cache(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens_k,
+                       const int32_t* page_table, int max_blocks_per_seq, int num_blocks, int cache_capacity, void* o,
+                       int o_dtype, float* lse, int B, int Nq, int Hq, int Hkv, int d, float scale, int causal,
+                       void* stream) {
+  if (!q || !k_cache || !v_cache || !seqlens_k || !o) return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Nq < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv) return ATTN_ERR_INVALID_ARG;
+  if (o_dtype != ATTN_F32 && o_dtype != ATTN_BF16) return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale) || (causal != 0 && causal != 1)) return ATTN_ERR_INVALID_ARG;
+  if (page_table) {
+    if (max_blocks_per_seq < 1 || num_blocks < 1) return ATTN_ERR_INVALID_ARG;
+    if ((long long)num_blocks * kPageTokens > INT32_MAX || (long long)max_blocks_per_seq * kPageTokens > INT32_MAX)
+      return ATTN_ERR_UNSUPPORTED;
+    if ((long long)max_blocks_per_seq * kPageTokens < Nq) return ATTN_ERR_INVALID_ARG;
+  } else {
+    if (cache_capacity < Nq) return ATTN_ERR_INVALID_ARG;
+  }
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
+  if ((long long)B * Nq * Hq > INT32_MAX) return ATTN_ERR_UNSUPPORTED;
+  unsigned* st = status_ptr();
+  if (!st) return ATTN_ERR_CUDA;
+  PrefillLaunch a;
+  a.q = q;
+  a.k = k_cache;
+  a.v = v_cache;
+  a.o = o;
+  a.o_bf16 = o_dtype == ATTN_BF16;
+  a.lse = lse;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.N = Nq;
+  a.d = d;
+  a.scale = scale;
+  a.causal = causal;
+  a.status = st;
+  a.seqlens = seqlens_k;
+  a.page_table = page_table;
+  a.capacity = cache_capacity;
+  a.max_blocks = max_blocks_per_seq;
+  a.num_blocks = num_blocks;
+  return cuda_status(launch_prefill(a, static_cast<cudaStream_t>(stream)), "attn_prefill_cache");
+}
+
 int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens_k,
                 const int32_t* page_table, int max_blocks_per_seq, int num_blocks, int cache_capacity,
                 int max_seqlen_k, void* o, int o_dtype, float* lse, int B, int T, int Hq, int Hkv, int d,

@@ -296,8 +296,9 @@ __global__ void __launch_bounds__(DecodeCfg<D, MT, FP8>::kThreads, DecodeCfg<D, 
       for (int kk = 0; kk < D / 16; ++kk) {
 #pragma unroll
         for (int nb = 0; nb < 2; ++nb) {
-          const uint32_t w = kw[nb][kk];
-          mma_f16_16816(sacc[nb], qa[kk], e4m3x2_to_f16x2(w), e4m3x2_to_f16x2(w >> 16));
+          uint32_t b0, b1;
+          e4m3x4_to_f16x2x2(kw[nb][kk], b0, b1);
+          mma_f16_16816(sacc[nb], qa[kk], b0, b1);
         }
       }
     }
@@ -416,10 +417,11 @@ __global__ void __launch_bounds__(DecodeCfg<D, MT, FP8>::kThreads, DecodeCfg<D, 
       for (int jj = 0; jj < D / 16; ++jj) {
         const int w = jj >> 1;
         const uint32_t sel = (jj & 1) ? 0x7362u : 0x5140u;
-        const uint32_t x01 = prmt(vw[0][w], vw[1][w], sel);
-        const uint32_t x23 = prmt(vw[2][w], vw[3][w], sel);
-        mma_f16_16816(o_acc[2 * jj], pa, e4m3x2_to_f16x2(x01), e4m3x2_to_f16x2(x23));
-        mma_f16_16816(o_acc[2 * jj + 1], pa, e4m3x2_to_f16x2(x01 >> 16), e4m3x2_to_f16x2(x23 >> 16));
+        uint32_t b01_j, b01_j1, b23_j, b23_j1;
+        e4m3x4_to_f16x2x2(prmt(vw[0][w], vw[1][w], sel), b01_j, b01_j1);
+        e4m3x4_to_f16x2x2(prmt(vw[2][w], vw[3][w], sel), b23_j, b23_j1);
+        mma_f16_16816(o_acc[2 * jj], pa, b01_j, b23_j);
+        mma_f16_16816(o_acc[2 * jj + 1], pa, b01_j1, b23_j1);
       }
     }
     __syncwarp();

@@ -41,15 +41,19 @@ struct DecodeLaunch {
 
 struct PrefillLaunch {
   const void* q;
-  const void* k;
+  const void* k;          // dense [B, N, Hkv, d], or a contiguous cache / paged pool
   const void* v;
   void* o;
   int o_bf16;
   float* lse;
-  int B, Hq, Hkv, N, d;
+  int B, Hq, Hkv, N, d;   // N: queries per sequence
   float scale;
   int causal;
   unsigned* status;
+  // prefill against an existing cache (seqlens == nullptr: dense K/V of N keys)
+  const int32_t* seqlens = nullptr;     // [B] keys per sequence, including the N new ones
+  const int32_t* page_table = nullptr;  // [B, max_blocks], or nullptr for a contiguous cache
+  int capacity = 0, max_blocks = 0, num_blocks = 0;
 };
 
 struct AppendLaunch {

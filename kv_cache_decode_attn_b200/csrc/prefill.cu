@@ -21,6 +21,15 @@
 // write out the previous item's O; the first PV of the new item waits until
 // that O has been read (O_FREE).
 //
+// Prefill against an existing cache (KV = contiguous or paged cache): the Nq
+// new queries of sequence b are its LAST Nq positions, so query row i sees keys
+// j <= L_b - Nq + i, where L_b = seqlens[b] counts the cached prefix plus the
+// Nq new keys (already appended).  Each item reads L_b, limits its K/V tiles to
+// the last key its rows see, and the softmax group that consumes a tile zeroes
+// the V rows at or past L_b in shared memory (cache rows there may hold any
+// bytes; paged blocks there are never loaded).  Paged caches load each 128-key
+// tile as eight 16-row boxes, one per physical block of the page table.
+//
 // Online softmax (running maximum m and denominator l per row, base-2 exponent
 // with the scale folded in): a row's reference maximum is only raised when the
 // tile maximum exceeds it by more than 8 (a factor 256), so O in TMEM is rescaled
@@ -32,7 +41,9 @@
 // "Numerical trick"; "大模型面試笔记——Attention篇" section 2 (online safe
 // softmax with the compensation factor); "[BEE-30062]" "背景" (FA2: scaling
 // moved out of the inner loop, parallel over query tiles; FA3: warp
-// specialisation with asynchronous TMA).
+// specialisation with asynchronous TMA); "Effizienz", "Der wichtige Maskenfehler
+// beim Cache" (queries aligned to the end of the key sequence) and the lesson's
+// "用它" (prefix caching) for the cached form.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -81,13 +92,21 @@ enum Bar {
   B_COUNT = 17
 };
 
+// Where K and V come from.
+enum KvSource { KV_DENSE = 0, KV_CACHE = 1, KV_PAGED = 2 };
+
 struct PrefillParams {
   void* o;
   float* lse;
   unsigned* status;
-  int B, N, Hq, Hkv, G, n_qblocks, n_ktiles, n_items;
+  int B, N, Hq, Hkv, G, n_qblocks, n_ktiles, n_items;   // N: queries per sequence (Nq)
   float scale_log2;
   int causal, o_bf16;
+  // cached forms only
+  const int32_t* seqlens;      // [B] keys per sequence, including the N new ones
+  const int32_t* page_table;   // [B, max_blocks] (paged)
+  int max_keys;                // cache capacity in tokens (contiguous) or max_blocks * 16 (paged)
+  int max_blocks, num_blocks;
 };
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
@@ -101,10 +120,13 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 
 struct Item {
   int qb, h, b, n_kv0, n_load;   // n_kv0: K/V tiles of query tile A; n_load: of tile B (>= n_kv0)
+  int L, off;                    // keys of the sequence; query row i sees keys j <= off + i (causal)
+  bool bad;                      // invalid length (cached forms): the rows are written as NaN
 };
 
 // Work item w: heaviest causal query blocks first, then consecutive heads (the
 // query heads of one K/V head are adjacent, so its K/V tiles are reused from L2).
+template <int KV>
 __device__ __forceinline__ Item item_of(int w, const PrefillParams& p) {
   Item it;
   const int per = p.Hq * p.B;
@@ -112,12 +134,26 @@ __device__ __forceinline__ Item item_of(int w, const PrefillParams& p) {
   const int r = w - (w / per) * per;
   it.h = r % p.Hq;
   it.b = r / p.Hq;
-  it.n_kv0 = p.causal ? min(2 * it.qb + 1, p.n_ktiles) : p.n_ktiles;
-  it.n_load = p.causal ? min(2 * it.qb + 2, p.n_ktiles) : p.n_ktiles;
+  if constexpr (KV == KV_DENSE) {
+    it.L = p.N;
+    it.off = 0;
+    it.bad = false;
+    it.n_kv0 = p.causal ? min(2 * it.qb + 1, p.n_ktiles) : p.n_ktiles;
+    it.n_load = p.causal ? min(2 * it.qb + 2, p.n_ktiles) : p.n_ktiles;
+  } else {
+    int L = __ldg(p.seqlens + it.b);
+    it.bad = L < p.N || L > p.max_keys;
+    if (it.bad) L = p.N;               // a safe stand-in; the host checked p.N <= p.max_keys
+    it.L = L;
+    it.off = L - p.N;
+    const int nt = (L + kBN - 1) / kBN;
+    it.n_kv0 = p.causal ? min((it.off + 2 * it.qb * kBM + kBM + kBN - 1) / kBN, nt) : nt;
+    it.n_load = p.causal ? min((it.off + 2 * it.qb * kBM + 2 * kBM + kBN - 1) / kBN, nt) : nt;
+  }
   return it;
 }
 
-template <int D>
+template <int D, int KV>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
@@ -167,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int last_g[2] = {-1, -1};
       bool ok = true;
       for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x, ++it) {
-        const Item itm = item_of(w, p);
+        const Item itm = item_of<KV>(w, p);
         const int kvh = itm.h / p.G;
         if (it > 0 && !wait_or_abort(&bars[B_QEMPTY], (it - 1) & 1, abort_flag, p.status)) break;
         mbar_arrive_expect_tx(&bars[B_QFULL], 2 * C::kTileBytes);
@@ -179,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_4d(smem + C::kQOff + t * C::kTileBytes + hh * C::kHalfBytes, &tmQ, &bars[B_QFULL], hh * 64,
                         itm.h, (2 * itm.qb + t) * kBM, itm.b, once);
         if (w + (int)gridDim.x < p.n_items) {       // warm L2 with the next item's Q
-          const Item nx = item_of(w + gridDim.x, p);
+          const Item nx = item_of<KV>(w + gridDim.x, p);
 #pragma unroll
           for (int t = 0; t < 2; ++t)
 #pragma unroll
@@ -192,16 +228,52 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           last_g[st] = g;
-          mbar_arrive_expect_tx(&bars[B_KFULL + st], C::kTileBytes);
+          if constexpr (KV != KV_PAGED) {
+            mbar_arrive_expect_tx(&bars[B_KFULL + st], C::kTileBytes);
 #pragma unroll
-          for (int hh = 0; hh < C::kHalves; ++hh)
-            tma_load_4d(smem + C::kKOff + st * C::kTileBytes + hh * C::kHalfBytes, &tmK, &bars[B_KFULL + st],
-                        hh * 64, kvh, t * kBN, itm.b, keep);
-          mbar_arrive_expect_tx(&bars[B_VFULL + st], C::kTileBytes);
+            for (int hh = 0; hh < C::kHalves; ++hh)
+              tma_load_4d(smem + C::kKOff + st * C::kTileBytes + hh * C::kHalfBytes, &tmK, &bars[B_KFULL + st],
+                          hh * 64, kvh, t * kBN, itm.b, keep);
+            mbar_arrive_expect_tx(&bars[B_VFULL + st], C::kTileBytes);
 #pragma unroll
-          for (int hh = 0; hh < C::kHalves; ++hh)
-            tma_load_4d(smem + C::kVOff + st * C::kTileBytes + hh * C::kHalfBytes, &tmV, &bars[B_VFULL + st],
-                        hh * 64, kvh, t * kBN, itm.b, keep);
+            for (int hh = 0; hh < C::kHalves; ++hh)
+              tma_load_4d(smem + C::kVOff + st * C::kTileBytes + hh * C::kHalfBytes, &tmV, &bars[B_VFULL + st],
+                          hh * 64, kvh, t * kBN, itm.b, keep);
+          } else {
+            // one 16-row box per physical block holding keys of this tile below L
+            constexpr int kBlocks = kBN / kPageTokens;
+            const int nb = min(kBlocks, (itm.L - t * kBN + kPageTokens - 1) / kPageTokens);
+            const int32_t* tab = p.page_table + (size_t)itm.b * p.max_blocks + t * kBlocks;
+            int ids[kBlocks];
+#pragma unroll
+            for (int jb = 0; jb < kBlocks; ++jb) {
+              int id = jb < nb ? __ldg(tab + jb) : 0;
+              if (id < 0 || id >= p.num_blocks) {
+                atomicOr(p.status, DEV_PAGE_ID);
+                id = 0;   // keep the byte count; the result is flagged invalid
+              }
+              ids[jb] = id;
+            }
+            const uint32_t bytes = nb * C::kHalves * kPageTokens * 128;
+            mbar_arrive_expect_tx(&bars[B_KFULL + st], bytes);
+#pragma unroll
+            for (int jb = 0; jb < kBlocks; ++jb) {
+              if (jb >= nb) break;
+#pragma unroll
+              for (int hh = 0; hh < C::kHalves; ++hh)
+                tma_load_3d(smem + C::kKOff + st * C::kTileBytes + hh * C::kHalfBytes + jb * kPageTokens * 128, &tmK,
+                            &bars[B_KFULL + st], hh * 64, kvh, ids[jb] * kPageTokens, keep);
+            }
+            mbar_arrive_expect_tx(&bars[B_VFULL + st], bytes);
+#pragma unroll
+            for (int jb = 0; jb < kBlocks; ++jb) {
+              if (jb >= nb) break;
+#pragma unroll
+              for (int hh = 0; hh < C::kHalves; ++hh)
+                tma_load_3d(smem + C::kVOff + st * C::kTileBytes + hh * C::kHalfBytes + jb * kPageTokens * 128, &tmV,
+                            &bars[B_VFULL + st], hh * 64, kvh, ids[jb] * kPageTokens, keep);
+            }
+          }
         }
       }
       // no copy may still be landing in shared memory when the CTA exits
@@ -238,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int pcnt[2] = {0, 0};                  // P_FULL phases consumed per tile
       bool ok = true;
       for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x, ++it) {
-        const Item itm = item_of(w, p);
+        const Item itm = item_of<KV>(w, p);
         const int g0 = g;
         ok = wait_or_abort(&bars[B_QFULL], it & 1, abort_flag, p.status) &&
              wait_or_abort(&bars[B_KFULL + (g0 & 1)], (g0 >> 1) & 1, abort_flag, p.status);
@@ -291,11 +363,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t s_addr = lane_base + C::s_col(t);
     const uint32_t o_addr = lane_base + C::o_col(t);
     int scnt = 0, it = 0;                               // S_FULL phases consumed, items done
+    int g_base = 0;                                     // K/V tiles of the previous items
     bool ok = true;
     for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x, ++it) {
-    const Item itm = item_of(w, p);
+    const Item itm = item_of<KV>(w, p);
     const int q_row = (2 * itm.qb + t) * kBM + row;
     const int nkv = t ? itm.n_load : itm.n_kv0;
+    const int g_item = g_base;
+    g_base += itm.n_load;
     float m = -INFINITY, l = 0.f;
     for (int j = 0; j < nkv; ++j) {
       if (!wait_or_abort(&bars[B_SFULL + t], (scnt++) & 1, abort_flag, p.status)) { ok = false; break; }
@@ -312,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // mask (causal diagonal tile, or keys past N) and the row maximum of the raw scores
       const int key0 = j * kBN;
-      const int lim = p.causal ? min(q_row - key0 + 1, p.N - key0) : (p.N - key0);   // visible keys: [0, lim)
+      const int lim = p.causal ? min(itm.off + q_row - key0 + 1, itm.L - key0) : (itm.L - key0);   // visible: [0, lim)
       if (lim < kBN) {
 #pragma unroll
         for (int c = 0; c < kBN; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
@@ -352,6 +427,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float ls = (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
       l = l * alpha + ls;
+      if constexpr (KV != KV_DENSE) {
+        // V rows of keys >= L: any bytes (cache) or never loaded (paged); the PV MMA
+        // would multiply them by p = 0.  The group that consumes the tile last zeroes
+        // them before its P arrives: tile A for j < n_kv0 (PV_A(j) is issued before
+        // PV_B(j)), tile B for the tiles only it reads.
+        const int valid = itm.L - key0;
+        if (valid < kBN && (warp & 3) == 0 && (t == 0 || j >= itm.n_kv0)) {
+          const int gj = g_item + j, st = gj & 1;
+          if (!wait_or_abort(&bars[B_VFULL + st], (gj >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+          uint8_t* vst = smem + C::kVOff + st * C::kTileBytes;
+          for (int idx = max(valid, 0) * 8 + lane; idx < kBN * 8; idx += 32)
+#pragma unroll
+            for (int hh = 0; hh < C::kHalves; ++hh)
+              *reinterpret_cast<uint4*>(vst + hh * C::kHalfBytes + idx * 16) = make_uint4(0, 0, 0, 0);
+          fence_proxy_async_smem();
+        }
+      }
       // O_t is stable here (PV_t(j-1) completed before S_t(j) did) and PV_t(j)
       // waits for this group's arrival below
       if (warp_raise && j > 0) {
@@ -378,7 +470,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     {
       tc_fence_after();
-      const float inv_l = 1.f / l;
+      const float inv_l = itm.bad ? __int_as_float(0x7fc00000) : 1.f / l;   // NaN rows for a bad length
+      if (itm.bad && t == 0 && row == 0) atomicOr(p.status, DEV_SEQLEN);
       const bool store = q_row < p.N;
       const size_t obase = (((size_t)itm.b * p.N + q_row) * p.Hq + itm.h) * D;
 #pragma unroll
@@ -407,7 +500,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (store && p.lse) p.lse[((size_t)itm.b * p.Hq + itm.h) * p.N + q_row] = (m + log2f(l)) * kLn2;
+      if (store && p.lse)
+        p.lse[((size_t)itm.b * p.Hq + itm.h) * p.N + q_row] = itm.bad ? __int_as_float(0x7fc00000) : (m + log2f(l)) * kLn2;
       // O_t has been read: the next item's first PV may overwrite it
       tc_fence_before();
       __syncwarp();
@@ -430,18 +524,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D>
+template <int D, int KV>
 cudaError_t run_prefill(const PrefillLaunch& a, cudaStream_t stream) {
   using C = PrefillCfg<D>;
   CUtensorMap tq, tk, tv;
-  // 4-D views {d, heads, N, B}; box {64, 1, 128, 1} with the 128-byte swizzle
-  auto enc = [&](CUtensorMap* m, const void* base, int heads) {
-    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)a.N, (cuuint64_t)a.B};
-    cuuint64_t str[3] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2, (cuuint64_t)a.N * heads * D * 2};
+  // 4-D views {d, heads, rows, B}; box {64, 1, 128, 1} with the 128-byte swizzle
+  auto enc = [&](CUtensorMap* m, const void* base, int heads, int rows) {
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)rows, (cuuint64_t)a.B};
+    cuuint64_t str[3] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2, (cuuint64_t)rows * heads * D * 2};
     cuuint32_t box[4] = {64, 1, (cuuint32_t)kBN, 1};
     return encode_tmap_nd(m, base, 4, dims, str, box);
   };
-  if (enc(&tq, a.q, a.Hq) || enc(&tk, a.k, a.Hkv) || enc(&tv, a.v, a.Hkv)) return cudaErrorInvalidValue;
+  if (enc(&tq, a.q, a.Hq, a.N)) return cudaErrorInvalidValue;
+  if constexpr (KV == KV_DENSE) {
+    if (enc(&tk, a.k, a.Hkv, a.N) || enc(&tv, a.v, a.Hkv, a.N)) return cudaErrorInvalidValue;
+  } else if constexpr (KV == KV_CACHE) {
+    if (enc(&tk, a.k, a.Hkv, a.capacity) || enc(&tv, a.v, a.Hkv, a.capacity)) return cudaErrorInvalidValue;
+  } else {
+    // pools [num_blocks, 16, Hkv, d] as {d, Hkv, num_blocks * 16}; one 16-row box per block
+    const uint64_t rows = (uint64_t)a.num_blocks * kPageTokens;
+    const uint64_t s1 = (uint64_t)D * 2, s2 = (uint64_t)a.Hkv * D * 2;
+    if (encode_tmap_3d(&tk, a.k, D, a.Hkv, rows, s1, s2, 64, 1, kPageTokens) ||
+        encode_tmap_3d(&tv, a.v, D, a.Hkv, rows, s1, s2, 64, 1, kPageTokens))
+      return cudaErrorInvalidValue;
+  }
   PrefillParams p;
   p.o = a.o;
   p.lse = a.lse;
@@ -459,7 +565,12 @@ cudaError_t run_prefill(const PrefillLaunch& a, cudaStream_t stream) {
   p.scale_log2 = a.scale * kLog2e;
   p.causal = a.causal;
   p.o_bf16 = a.o_bf16;
-  auto kern = prefill_kernel<D>;
+  p.seqlens = a.seqlens;
+  p.page_table = a.page_table;
+  p.max_blocks = a.max_blocks;
+  p.num_blocks = a.num_blocks;
+  p.max_keys = KV == KV_PAGED ? a.max_blocks * kPageTokens : (KV == KV_CACHE ? a.capacity : a.N);
+  auto kern = prefill_kernel<D, KV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   // persistent: one CTA per SM (each owns all 512 TMEM columns)
@@ -474,7 +585,10 @@ cudaError_t run_prefill(const PrefillLaunch& a, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_prefill(const PrefillLaunch& a, cudaStream_t stream) {
-  return a.d == 128 ? run_prefill<128>(a, stream) : run_prefill<64>(a, stream);
+  if (!a.seqlens) return a.d == 128 ? run_prefill<128, KV_DENSE>(a, stream) : run_prefill<64, KV_DENSE>(a, stream);
+  if (!a.page_table)
+    return a.d == 128 ? run_prefill<128, KV_CACHE>(a, stream) : run_prefill<64, KV_CACHE>(a, stream);
+  return a.d == 128 ? run_prefill<128, KV_PAGED>(a, stream) : run_prefill<64, KV_PAGED>(a, stream);
 }
 
 }  // namespace kvattn

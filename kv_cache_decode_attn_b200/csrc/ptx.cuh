@@ -173,6 +173,17 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
   return d;
 }
 
+// Four e4m3 codes (bytes 0..3 of w) to two f16 pairs: lo = bytes 0, 1 and hi =
+// bytes 2, 3, taken straight from the register halves.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\t"
+      "mov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
+}
+
 // Two f32 values to two e4m3 codes (lo -> low byte), round to nearest even,
 // saturating to +-448 (NaN stays NaN).
 __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {

@@ -139,6 +139,28 @@ def test_append_fp8_rejects_bad_arguments():
     assert L.kv_append_fp8(P, P, P, P, P, P, P, None, 0, 0, 10, 1, 1, 2, 96, None) == kv.ATTN_ERR_UNSUPPORTED
 
 
+def test_prefill_cache_rejects_bad_arguments():
+    L = kv.lib
+
+    def call(**kw):
+        a = dict(q=P, k=P, v=P, sl=P, pt=None, mb=0, nb=0, cap=100, o=P, od=0, lse=None, B=2, Nq=10, Hq=8, Hkv=2,
+                 d=128, scale=0.1, causal=1)
+        a.update(kw)
+        return L.attn_prefill_cache(a["q"], a["k"], a["v"], a["sl"], a["pt"], a["mb"], a["nb"], a["cap"], a["o"],
+                                    a["od"], a["lse"], a["B"], a["Nq"], a["Hq"], a["Hkv"], a["d"], a["scale"],
+                                    a["causal"], None)
+
+    assert call(sl=None) == kv.ATTN_ERR_INVALID_ARG
+    assert call(Nq=0) == kv.ATTN_ERR_INVALID_ARG
+    assert call(Hkv=3) == kv.ATTN_ERR_INVALID_ARG
+    assert call(cap=9) == kv.ATTN_ERR_INVALID_ARG             # capacity below Nq
+    assert call(pt=P, mb=0, nb=4) == kv.ATTN_ERR_INVALID_ARG
+    assert call(pt=P, mb=1, nb=4, Nq=17) == kv.ATTN_ERR_INVALID_ARG   # 16 slots for 17 queries
+    assert call(d=96) == kv.ATTN_ERR_UNSUPPORTED
+    assert call(od=3) == kv.ATTN_ERR_INVALID_ARG
+    assert call(q=P + 4) == kv.ATTN_ERR_INVALID_ARG
+
+
 def test_binding_checks_fp8_cache_dtype():
     import torch
     x = torch.zeros(1, 4, 2, 128, dtype=torch.bfloat16)
