@@ -58,7 +58,8 @@ enum {
   ATTN_ERR_UNSUPPORTED = -2, /* valid request outside what is built (d, rows per KV head) */
   ATTN_ERR_WORKSPACE = -3,   /* decode workspace missing or smaller than required */
   ATTN_ERR_CUDA = -4,        /* a CUDA runtime/driver call failed (launch, tensor map, ...) */
-  ATTN_ERR_DEVICE = -5       /* the device status word is non-zero (attn_get_device_status) */
+  ATTN_ERR_DEVICE = -5,      /* the device status word is non-zero (attn_get_device_status) */
+  ATTN_ERR_NO_BLOCKS = -6    /* the block pool cannot meet the request (nothing was changed) */
 };
 
 /* ---- output element types ------------------------------------------------ */
@@ -298,6 +299,110 @@ ATTN_API int attn_decode_noalloc(const void* q, const void* k_cache, const void*
 
 /* attn_status_string -- static text for a return code (never NULL). */
 ATTN_API const char* attn_status_string(int status);
+
+/*
+ * ------------------------------------------------------------------ block pool
+ * Host-side allocator of the 16-token physical blocks of a paged KV cache.
+ *
+ * Defines: [P1] "页面注意 KV缓存作为虚拟内存" (the cache is cut into fixed
+ * 16-token blocks; a page table maps logical positions to physical blocks;
+ * blocks are shared between parallel samples and reused prefixes) and its
+ * exercises 2 (prefix caching: fill the cache for a prompt once, then branch
+ * per completion) and 3 (a finished sequence returns its blocks to the pool).
+ * Not on the device path: the pool only hands out block ids; the caller writes
+ * the tables it produces into device memory for kv_append / attn_decode /
+ * attn_prefill_cache.  Every call is thread-safe (one mutex per pool) and
+ * all-or-nothing: a request that cannot be met returns a negative status and
+ * changes nothing.  Free blocks form a LIFO stack with block 0 on top at
+ * creation; a freed sequence pushes its blocks last-to-first.
+ */
+typedef struct attn_block_pool attn_block_pool;
+
+/* A pool of num_blocks blocks of block_tokens tokens (16 for the kernels).
+ * NULL if an argument is < 1 or memory runs out.  Owned by the caller. */
+ATTN_API attn_block_pool* attn_block_pool_create(int num_blocks, int block_tokens);
+ATTN_API void attn_block_pool_destroy(attn_block_pool* pool);
+/* Blocks not referenced by any sequence. */
+ATTN_API int attn_block_pool_free_blocks(attn_block_pool* pool);
+/* Sequences that reference a block (0 = free). */
+ATTN_API int attn_block_ref_count(attn_block_pool* pool, int32_t block);
+/* A new empty sequence; returns its id (>= 0; the smallest freed id is reused first). */
+ATTN_API int attn_seq_create(attn_block_pool* pool);
+/* A new sequence sharing every block of `parent` (reference counts + 1), same length. */
+ATTN_API int attn_seq_fork(attn_block_pool* pool, int parent);
+/* Room for n_new more tokens at positions length .. length + n_new - 1.  If the
+ * sequence's last block is partly filled and shared with another sequence, it is
+ * first replaced by a private block: *n_cow = 1 and (*cow_src, *cow_dst) name the
+ * block whose contents the caller must copy (attn_copy_blocks) before writing;
+ * else *n_cow = 0.  Then the blocks the new length needs are taken.
+ * ATTN_ERR_NO_BLOCKS if the pool is short (nothing changed). */
+ATTN_API int attn_seq_reserve(attn_block_pool* pool, int seq, int n_new, int32_t* cow_src, int32_t* cow_dst,
+                              int* n_cow);
+/* Release a sequence: each of its blocks loses one reference; unreferenced blocks return to the pool. */
+ATTN_API int attn_seq_free(attn_block_pool* pool, int seq);
+/* Tokens the sequence holds (reserved so far). */
+ATTN_API int64_t attn_seq_length(attn_block_pool* pool, int seq);
+/* The sequence's physical block ids in logical order into out[capacity] (out may be
+ * NULL to ask for the count); returns the number of blocks. */
+ATTN_API int attn_seq_block_table(attn_block_pool* pool, int seq, int32_t* out, int capacity);
+/* Host page table [n_seqs, max_blocks] (row i = seqs[i]'s blocks, -1 padded) and
+ * int32 lengths [n_seqs] (lens may be NULL): the page_table / seqlens layout the
+ * kernels read.  ATTN_ERR_INVALID_ARG if a sequence needs more than max_blocks. */
+ATTN_API int attn_block_pool_page_table(attn_block_pool* pool, const int32_t* seqs, int n_seqs, int max_blocks,
+                                        int32_t* table, int32_t* lens);
+
+/*
+ * attn_copy_blocks -- device copy of whole blocks of both pools, src[i] -> dst[i]
+ * (the copy-on-write step above).  k_pool, v_pool: device [num_blocks, 16, Hkv, d]
+ * with elem_bytes 2 (bf16) or 1 (e4m3); src, dst: device int32 [n], n <= 65535.
+ * Ids outside [0, num_blocks) are skipped and set ATTN_DEV_PAGE_ID.  A pair must
+ * not have its destination used as another pair's source in the same call.
+ */
+ATTN_API int attn_copy_blocks(void* k_pool, void* v_pool, const int32_t* src, const int32_t* dst, int n,
+                              int num_blocks, int Hkv, int d, int elem_bytes, void* stream);
+
+/*
+ * attn_pool_simulate -- paged versus contiguous KV memory over a request trace
+ * ([P1] exercise 3: many chat completions of different lengths, blocks returned
+ * to the pool when a sequence finishes; compare the fragmentation with
+ * contiguous allocation).  Host only.
+ *
+ * events: n_events triples (op, request, n): op 0 = the request starts holding n
+ * tokens (its prompt), 1 = it grows by n tokens, 2 = it finishes.  Both
+ * allocators see every event and an arena of arena_tokens tokens:
+ *   paged       a block pool of arena_tokens / block_tokens blocks (attn_seq_*);
+ *               a start that cannot get its blocks is rejected, a growth that
+ *               cannot is dropped (its blocks are released, later events ignored);
+ *   contiguous  every started request reserves reserve_tokens consecutive tokens
+ *               (the worst-case length), or with reserve_tokens = 0 exactly its
+ *               final length (the sum of its start and growth tokens in the
+ *               trace; at least 1); first fit over the free extents, which
+ *               merge when released; a start that finds no extent is rejected,
+ *               a growth beyond the reservation is dropped.
+ * After every event: reserved tokens (paged: blocks held x block_tokens;
+ * contiguous: reservations held), stored tokens (lengths of live requests), and
+ * for contiguous the free tokens outside the largest free extent (external
+ * fragmentation).  metrics[ATTN_SIM_METRICS] receives, per allocator: rejected
+ * starts, dropped requests, peak reserved tokens, and the sums over events of
+ * reserved and of stored tokens (utilisation = stored sum / reserved sum), plus
+ * the contiguous external-fragmentation sum.
+ */
+enum {
+  ATTN_SIM_PAGED_REJECTED = 0,
+  ATTN_SIM_PAGED_DROPPED = 1,
+  ATTN_SIM_PAGED_PEAK_RESERVED = 2,
+  ATTN_SIM_PAGED_SUM_RESERVED = 3,
+  ATTN_SIM_PAGED_SUM_STORED = 4,
+  ATTN_SIM_CONTIG_REJECTED = 5,
+  ATTN_SIM_CONTIG_DROPPED = 6,
+  ATTN_SIM_CONTIG_PEAK_RESERVED = 7,
+  ATTN_SIM_CONTIG_SUM_RESERVED = 8,
+  ATTN_SIM_CONTIG_SUM_STORED = 9,
+  ATTN_SIM_CONTIG_SUM_EXTERNAL = 10,
+  ATTN_SIM_METRICS = 11
+};
+ATTN_API int attn_pool_simulate(const int32_t* events, int n_events, int64_t arena_tokens, int block_tokens,
+                                int64_t reserve_tokens, int64_t* metrics);
 
 #ifdef __cplusplus
 }

@@ -21,7 +21,8 @@ import torch
 __all__ = [
     "lib", "LIB_PATH", "AttnError",
     "attn_prefill", "attn_decode", "attn_decode_workspace_bytes", "attn_decode_noalloc", "kv_append",
-    "attn_decode_fp8", "kv_append_fp8", "attn_prefill_cache",
+    "attn_decode_fp8", "kv_append_fp8", "attn_prefill_cache", "BlockPool", "copy_blocks", "pool_simulate",
+    "ATTN_ERR_NO_BLOCKS", "SIM_METRICS",
     "kv_cache_bytes", "ATTN_DECODE_NOALLOC_SCRATCH_BYTES",
     "attn_get_device_status", "attn_status_string", "decode_workspace",
     "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_WORKSPACE", "ATTN_ERR_CUDA",
@@ -32,6 +33,11 @@ __all__ = [
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvattn.so")
 
 ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_WORKSPACE, ATTN_ERR_CUDA, ATTN_ERR_DEVICE = 0, -1, -2, -3, -4, -5
+ATTN_ERR_NO_BLOCKS = -6
+# attn_pool_simulate's metrics, in the order of the ATTN_SIM_* indices
+SIM_METRICS = ["paged_rejected", "paged_dropped", "paged_peak_reserved", "paged_sum_reserved", "paged_sum_stored",
+               "contig_rejected", "contig_dropped", "contig_peak_reserved", "contig_sum_reserved", "contig_sum_stored",
+               "contig_sum_external"]
 ATTN_F32, ATTN_BF16 = 0, 1
 ATTN_DECODE_NOALLOC_SCRATCH_BYTES = 32 << 20
 ATTN_DEV_PAGE_ID, ATTN_DEV_SEQLEN, ATTN_DEV_APPEND_RANGE, ATTN_DEV_TIMEOUT, ATTN_DEV_SCALE = 1, 2, 4, 8, 16
@@ -51,6 +57,19 @@ _SIGNATURES = {
     "kv_append": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p]),
     "kv_append_fp8": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p]),
     "kv_cache_bytes": (_i64, [_i, _i, _i64, _i, _i, _i]),
+    "attn_block_pool_create": (_p, [_i, _i]),
+    "attn_block_pool_destroy": (None, [_p]),
+    "attn_block_pool_free_blocks": (_i, [_p]),
+    "attn_block_ref_count": (_i, [_p, ctypes.c_int32]),
+    "attn_seq_create": (_i, [_p]),
+    "attn_seq_fork": (_i, [_p, _i]),
+    "attn_seq_reserve": (_i, [_p, _i, _i, _p, _p, _p]),
+    "attn_seq_free": (_i, [_p, _i]),
+    "attn_seq_length": (_i64, [_p, _i]),
+    "attn_seq_block_table": (_i, [_p, _i, _p, _i]),
+    "attn_block_pool_page_table": (_i, [_p, _p, _i, _i, _p, _p]),
+    "attn_copy_blocks": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _p]),
+    "attn_pool_simulate": (_i, [_p, _i, _i64, _i, _i64, _p]),
     "attn_get_device_status": (_i, [_i]),
     "attn_status_string": (ctypes.c_char_p, [_i]),
 }
@@ -285,3 +304,99 @@ def kv_cache_bytes(n_layers, batch, tokens, n_kv_heads, head_dim, elem_bytes) ->
 
 def attn_get_device_status(clear: bool = False) -> int:
     return int(lib.attn_get_device_status(int(bool(clear))))
+
+
+# ------------------------------------------------------------------ block pool
+class BlockPool:
+    """Host allocator of 16-token KV blocks (``attn_block_pool_*`` / ``attn_seq_*``).
+
+    ``reserve`` returns the copy-on-write pairs ``[(src, dst)]`` the caller must
+    copy on the device (``copy_blocks``) before writing the new tokens.
+    """
+
+    def __init__(self, num_blocks: int, block_tokens: int = 16):
+        self._h = lib.attn_block_pool_create(int(num_blocks), int(block_tokens))
+        if not self._h:
+            raise AttnError("attn_block_pool_create", ATTN_ERR_INVALID_ARG)
+        self.num_blocks, self.block_tokens = int(num_blocks), int(block_tokens)
+
+    def close(self) -> None:
+        if self._h:
+            lib.attn_block_pool_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @staticmethod
+    def _ok(fn: str, st: int) -> int:
+        if st < 0:
+            raise AttnError(fn, st)
+        return st
+
+    def free_blocks(self) -> int:
+        return self._ok("attn_block_pool_free_blocks", lib.attn_block_pool_free_blocks(self._h))
+
+    def ref_count(self, block: int) -> int:
+        return self._ok("attn_block_ref_count", lib.attn_block_ref_count(self._h, int(block)))
+
+    def create(self) -> int:
+        return self._ok("attn_seq_create", lib.attn_seq_create(self._h))
+
+    def fork(self, parent: int) -> int:
+        return self._ok("attn_seq_fork", lib.attn_seq_fork(self._h, int(parent)))
+
+    def reserve(self, seq: int, n_new: int) -> list[tuple[int, int]]:
+        src, dst, n = ctypes.c_int32(0), ctypes.c_int32(0), ctypes.c_int(0)
+        self._ok("attn_seq_reserve", lib.attn_seq_reserve(self._h, int(seq), int(n_new), ctypes.byref(src),
+                                                          ctypes.byref(dst), ctypes.byref(n)))
+        return [(src.value, dst.value)] if n.value else []
+
+    def free(self, seq: int) -> None:
+        self._ok("attn_seq_free", lib.attn_seq_free(self._h, int(seq)))
+
+    def length(self, seq: int) -> int:
+        return self._ok("attn_seq_length", lib.attn_seq_length(self._h, int(seq)))
+
+    def blocks(self, seq: int) -> list[int]:
+        n = self._ok("attn_seq_block_table", lib.attn_seq_block_table(self._h, int(seq), None, 0))
+        out = (ctypes.c_int32 * max(n, 1))()
+        self._ok("attn_seq_block_table", lib.attn_seq_block_table(self._h, int(seq), out, n))
+        return list(out[:n])
+
+    def page_table(self, seqs, max_blocks: int):
+        """Host int32 page table ``[len(seqs), max_blocks]`` (-1 padded) and lengths, as torch tensors."""
+        seqs = torch.as_tensor(list(seqs), dtype=torch.int32)
+        table = torch.empty(len(seqs), int(max_blocks), dtype=torch.int32)
+        lens = torch.empty(len(seqs), dtype=torch.int32)
+        self._ok("attn_block_pool_page_table",
+                 lib.attn_block_pool_page_table(self._h, seqs.data_ptr(), len(seqs), int(max_blocks),
+                                                table.data_ptr(), lens.data_ptr()))
+        return table, lens
+
+
+def copy_blocks(k_pool, v_pool, src, dst, stream=None) -> None:
+    """Copy whole blocks src[i] -> dst[i] of both device pools ``[nblk, 16, Hkv, d]``
+    (bf16, or e4m3 codes); src/dst device int32 ``[n]``."""
+    if tuple(v_pool.shape) != tuple(k_pool.shape) or src.shape != dst.shape:
+        raise ValueError("shape mismatch")
+    nblk, _, Hkv, d = k_pool.shape
+    st = lib.attn_copy_blocks(_dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"), _dev(src, "src", torch.int32),
+                              _dev(dst, "dst", torch.int32), int(src.numel()), int(nblk), int(Hkv), int(d),
+                              int(k_pool.element_size()), _stream(stream))
+    _check("attn_copy_blocks", st)
+
+
+def pool_simulate(events, arena_tokens: int, block_tokens: int = 16, reserve_tokens: int = 0) -> dict:
+    """``attn_pool_simulate`` over an int32 ``[n, 3]`` (op, request, n) trace; returns the metrics by name."""
+    ev = torch.as_tensor(events, dtype=torch.int32).contiguous().view(-1)
+    if ev.numel() % 3:
+        raise ValueError("events must be triples")
+    out = torch.zeros(len(SIM_METRICS), dtype=torch.int64)
+    st = lib.attn_pool_simulate(ev.data_ptr(), ev.numel() // 3, int(arena_tokens), int(block_tokens),
+                                int(reserve_tokens), out.data_ptr())
+    _check("attn_pool_simulate", st)
+    return dict(zip(SIM_METRICS, (int(x) for x in out)))

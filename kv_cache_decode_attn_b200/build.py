@@ -1,7 +1,7 @@
 """Build ``libkvattn.so`` in-tree with nvcc for sm_100a.
 
 ``python kv_cache_decode_attn_b200/build.py`` (or ``build()``) compiles every
-``csrc/*.cu`` file into one shared library beside this file.  The library links
+``csrc/*.cu`` and ``csrc/*.cpp`` file into one shared library beside this file.  The library links
 the CUDA runtime statically and reaches the driver API (tensor-map encoding)
 through ``cudaGetDriverEntryPointByVersion``, so it needs no ``-lcuda`` at link
 time.  Rebuilds only when a source is newer than the library.
@@ -33,7 +33,8 @@ def _nvcc() -> str:
 
 
 def sources() -> list[str]:
-    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    # CUDA sources and the host-only C++ sources (nvcc hands .cpp files to the host compiler)
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
 
 
 def _stale() -> bool:

@@ -119,6 +119,7 @@ const char* attn_status_string(int status) {
     case ATTN_ERR_WORKSPACE: return "workspace missing or too small";
     case ATTN_ERR_CUDA: return "CUDA error";
     case ATTN_ERR_DEVICE: return "device-side error flagged";
+    case ATTN_ERR_NO_BLOCKS: return "block pool exhausted";
     default: return "unknown status";
   }
 }
@@ -360,6 +361,23 @@ int kv_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new
               int Hkv, int d, void* stream) {
   return append_impl(k_cache, v_cache, k_new, v_new, nullptr, nullptr, false, cache_lens, page_table,
                      max_blocks_per_seq, num_blocks, cache_capacity, B, T, Hkv, d, stream, "kv_append");
+}
+
+int attn_copy_blocks(void* k_pool, void* v_pool, const int32_t* src, const int32_t* dst, int n, int num_blocks,
+                     int Hkv, int d, int elem_bytes, void* stream) {
+  if (!k_pool || !v_pool || n < 0 || num_blocks < 1 || Hkv < 1) return ATTN_ERR_INVALID_ARG;
+  if (n > 0 && (!src || !dst)) return ATTN_ERR_INVALID_ARG;
+  if (n > 65535) return ATTN_ERR_UNSUPPORTED;
+  if ((d != 64 && d != 128) || (elem_bytes != 1 && elem_bytes != 2)) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(k_pool) || !aligned16(v_pool)) return ATTN_ERR_INVALID_ARG;
+  if (n == 0) return ATTN_OK;
+  const long long block_bytes = (long long)kPageTokens * Hkv * d * elem_bytes;
+  if (block_bytes / 16 > INT32_MAX) return ATTN_ERR_UNSUPPORTED;
+  unsigned* st = status_ptr();
+  if (!st) return ATTN_ERR_CUDA;
+  return cuda_status(launch_copy_blocks(k_pool, v_pool, src, dst, n, num_blocks, (int)block_bytes, st,
+                                        static_cast<cudaStream_t>(stream)),
+                     "attn_copy_blocks");
 }
 
 int kv_append_fp8(void* k_cache, void* v_cache, const void* k_new, const void* v_new, const float* k_scale,

@@ -101,5 +101,8 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream);
 cudaError_t launch_decode_tc(const DecodeLaunch& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream);
 cudaError_t launch_append(const AppendLaunch& a, cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillLaunch& a, cudaStream_t stream);
+// copy n whole blocks (src[i] -> dst[i], device id lists) of both pools
+cudaError_t launch_copy_blocks(void* k, void* v, const int32_t* src, const int32_t* dst, int n, int num_blocks,
+                               int block_bytes, unsigned* status, cudaStream_t stream);
 
 }  // namespace kvattn

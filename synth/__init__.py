@@ -21,6 +21,10 @@ Recipe (the same on every machine with the same torch build):
   cast of seeded N(0, 1) draws divided by the head's scale (clamped to +-448),
   so that the dequantised cache is again about N(0, 1).  The library's own
   quantiser (the FP8 append path) is not involved in making inputs.
+* Request traces (block-pool simulation): prompt and output lengths uniform
+  on closed intervals (PCG64); at most ``max_live`` requests at once, each
+  growing by ``grow_step`` tokens per step until its output is complete, new
+  requests starting (in index order) as soon as a slot frees.
 * Seeds: ``1000 + index`` of the workload in ``WORKLOADS`` unless a test
   chooses its own.
 """
@@ -220,3 +224,33 @@ def workload_decode(name: str, device="cpu", **kw) -> tuple[Decode, DecodeCase]:
     w = WORKLOADS[name]
     return w, decode_inputs(w.B, w.T, w.Hq, w.Hkv, w.d, w.len_lo, w.len_hi, SEEDS[name],
                             device=device, paged=w.paged, fp8=w.fp8, **kw)
+
+
+def request_trace(n_requests: int, max_live: int, prompt_lo: int, prompt_hi: int, out_lo: int, out_hi: int,
+                  grow_step: int, seed: int) -> np.ndarray:
+    """int32 [n_events, 3] trace of (op, request, n): op 0 = start with its prompt,
+    1 = grow by n tokens, 2 = finish.  Chat completions of different lengths, at
+    most ``max_live`` at a time, every live request growing ``grow_step`` tokens
+    per step."""
+    rng = np.random.Generator(np.random.PCG64(int(seed)))
+    prompts = rng.integers(prompt_lo, prompt_hi + 1, size=n_requests)
+    outputs = rng.integers(out_lo, out_hi + 1, size=n_requests)
+    events, live, nxt = [], [], 0
+    left = {}
+    while nxt < n_requests or live:
+        while len(live) < max_live and nxt < n_requests:
+            events.append((0, nxt, int(prompts[nxt])))
+            left[nxt] = int(outputs[nxt])
+            live.append(nxt)
+            nxt += 1
+        still = []
+        for r in live:
+            n = min(grow_step, left[r])
+            events.append((1, r, n))
+            left[r] -= n
+            if left[r] == 0:
+                events.append((2, r, 0))
+            else:
+                still.append(r)
+        live = still
+    return np.asarray(events, dtype=np.int32)
