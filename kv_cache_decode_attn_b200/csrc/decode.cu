@@ -34,6 +34,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "split.cuh"
 
 namespace kvattn {
 namespace {
@@ -60,28 +61,6 @@ struct DecodeCfg {
   static constexpr int kSmemBytes = kStatsOffset + MT * 4 * 16 * 2 * 4 + 16 + 1024;  // + alignment slack
   static constexpr int kMinBlocks = (kSmemBytes * 2 <= 227 * 1024) ? 2 : 1;
 };
-
-struct SplitParams {
-  const __nv_bfloat16* q;
-  const float* k_scale;   // FP8 caches: per-KV-head scales (else unused)
-  const float* v_scale;
-  const int32_t* seqlens;
-  const int32_t* page_table;
-  float* part_o;
-  float* part_lse;
-  unsigned* status;
-  int T, Hq, Hkv, G, R;
-  int chunk, max_chunks, capacity, max_blocks, num_blocks, max_seqlen;
-  float scale_log2;
-  int causal;
-};
-
-__device__ __forceinline__ bool seqlen_bad(int L, int T, int max_seqlen, bool paged, int capacity, int max_blocks) {
-  if (L < T || L > max_seqlen) return true;
-  if (!paged && L > capacity) return true;
-  if (paged && (L + kPageTokens - 1) / kPageTokens > max_blocks) return true;
-  return false;
-}
 
 // bf16 pair (low = lower index) -> f16 pair
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
@@ -138,57 +117,8 @@ __global__ void __launch_bounds__(DecodeCfg<D, MT, FP8>::kThreads, DecodeCfg<D, 
 
   if (warp == C::kConsumerWarps) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
-      const uint64_t pol = policy_evict_first();
-      for (int i = 0; i < n_tiles; ++i) {
-        const int s = i % C::kStages;
-        if (i >= C::kStages && !mbar_wait(&empty[s], ((i / C::kStages) - 1) & 1)) {
-          atomicOr(p.status, DEV_TIMEOUT);
-          *reinterpret_cast<volatile int*>(abort_flag) = 1;
-          break;
-        }
-        uint8_t* kst = smem + s * C::kStageBytes;
-        uint8_t* vst = kst + C::kTensorBytes;
-        const int t0 = tok_begin + i * kDecodeTile;
-        if (!PAGED) {
-          mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-          const int row = b * p.capacity + t0;
-#pragma unroll
-          for (int h = 0; h < C::kHalves; ++h) {
-            tma_load_3d(kst + h * C::kHalfBytes, &tmK, &full[s], h * 64, g, row, pol);
-            tma_load_3d(vst + h * C::kHalfBytes, &tmV, &full[s], h * 64, g, row, pol);
-          }
-        } else {
-          constexpr int kBlocks = kDecodeTile / kPageTokens;
-          const int nb = min(kBlocks, (tok_end - t0 + kPageTokens - 1) / kPageTokens);
-          const int32_t* row_tab = p.page_table + (size_t)b * p.max_blocks + t0 / kPageTokens;
-          // read the stage's block ids together: the copies' memory clobbers would
-          // otherwise serialise one table read per block
-          int ids[kBlocks];
-#pragma unroll
-          for (int j = 0; j < kBlocks; ++j) ids[j] = j < nb ? __ldg(row_tab + j) : 0;
-          mbar_arrive_expect_tx(&full[s], nb * 2 * C::kHalves * kPageTokens * 128);
-#pragma unroll
-          for (int j = 0; j < kBlocks; ++j) {
-            if (j >= nb) break;
-            int blk = ids[j];
-            if (blk < 0 || blk >= p.num_blocks) {
-              atomicOr(p.status, DEV_PAGE_ID);
-              blk = 0;   // keep the byte count; the result is flagged invalid
-            }
-#pragma unroll
-            for (int h = 0; h < C::kHalves; ++h) {
-              tma_load_3d(kst + h * C::kHalfBytes + j * kPageTokens * 128, &tmK, &full[s], h * 64, g,
-                          blk * kPageTokens, pol);
-              tma_load_3d(vst + h * C::kHalfBytes + j * kPageTokens * 128, &tmV, &full[s], h * 64, g,
-                          blk * kPageTokens, pol);
-            }
-          }
-        }
-      }
-    }
+    if (lane == 0) produce_split_tiles<C, PAGED>(smem, full, empty, &tmK, &tmV, p, b, g, tok_begin, tok_end, n_tiles,
+                                                abort_flag);
     return;
   }
 
@@ -681,7 +611,8 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
   cudaError_t e;
   if (a.fp8) {
     // api.cu admits d == 128 and at most kDecodeMmaRows rows per KV head
-    if (R <= 16) e = paged ? run_split<128, 1, true, true>(tk, tv, sp, a.B, stream)
+    if (R <= 8) e = launch_decode_fp8_rows8(tk, tv, sp, a.B, paged, stream);
+    else if (R <= 16) e = paged ? run_split<128, 1, true, true>(tk, tv, sp, a.B, stream)
                            : run_split<128, 1, false, true>(tk, tv, sp, a.B, stream);
     else e = paged ? run_split<128, 2, true, true>(tk, tv, sp, a.B, stream)
                    : run_split<128, 2, false, true>(tk, tv, sp, a.B, stream);

@@ -86,8 +86,9 @@ def test_fp8_decode_small_parity(paged, T, Hq, Hkv):
 
 @pytest.mark.parametrize("num_splits", [1, 3, 16])
 @pytest.mark.parametrize("causal", [True, False])
-def test_fp8_split_counts_noncausal_bf16_out(num_splits, causal):
-    T, Hq, Hkv, d = 4, 16, 4, 128
+@pytest.mark.parametrize("T,Hq,Hkv", [(4, 16, 4), (2, 8, 2)])     # 16 rows per KV head; 8 (transposed kernel)
+def test_fp8_split_counts_noncausal_bf16_out(num_splits, causal, T, Hq, Hkv):
+    d = 128
     lens = [5, 700, 4100]
     case = synth.decode_inputs(len(lens), T, Hq, Hkv, d, 0, 0, seed=77, device="cuda", lengths=lens, fp8=True)
     host = host_copy(case)
@@ -144,8 +145,9 @@ def test_fp8_append_is_bit_exact(paged, d):
     assert np.array_equal(vg, vr)
 
 
-def test_fp8_decode_ignores_nan_codes_past_the_end():
-    T, Hq, Hkv, d = 2, 16, 2, 128
+@pytest.mark.parametrize("T,Hq,Hkv", [(2, 16, 2), (1, 16, 2)])
+def test_fp8_decode_ignores_nan_codes_past_the_end(T, Hq, Hkv):
+    d = 128
     lens = [3, 64, 100, 511]
     for paged in (False, True):
         case = synth.decode_inputs(len(lens), T, Hq, Hkv, d, 0, 0, seed=9, device="cuda", paged=paged,
@@ -169,8 +171,9 @@ def test_fp8_decode_ignores_nan_codes_past_the_end():
         check_lse(lse, lse_ref)
 
 
-def test_fp8_paged_equals_contiguous_bitwise():
-    T, Hq, Hkv, d = 4, 32, 4, 128
+@pytest.mark.parametrize("T,Hq,Hkv", [(4, 32, 4), (2, 16, 4)])
+def test_fp8_paged_equals_contiguous_bitwise(T, Hq, Hkv):
+    d = 128
     lens = [1, 77, 1000, 4000]
     cont = synth.decode_inputs(len(lens), T, Hq, Hkv, d, 0, 0, seed=21, device="cuda", lengths=lens, fp8=True)
     paged = synth.decode_inputs(len(lens), T, Hq, Hkv, d, 0, 0, seed=21, device="cuda", lengths=lens, paged=True,
