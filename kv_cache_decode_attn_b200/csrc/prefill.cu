@@ -1,7 +1,9 @@
 // Prefill attention on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
 //
-// Persistent: one CTA per SM walks a list of work items, heaviest causal query
-// blocks first.  A work item is two 128-row query tiles (A: rows 256*qb .. +127,
+// Persistent: one CTA per SM takes work items from a queue, heaviest causal
+// query blocks first (its first item is its block index; every further item is
+// a ticket from a global counter, so a CTA that finishes early takes more
+// work instead of waiting on a fixed share).  A work item is two 128-row query tiles (A: rows 256*qb .. +127,
 // B: the next 128) of one (batch, query head); both tiles share every K/V tile
 // loaded for the item.  Warp roles:
 //   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread i of a
@@ -47,10 +49,21 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "internal.h"
 #include "ptx.cuh"
 
 namespace kvattn {
+
+// Work-queue counters of the prefill kernel: slot i holds (next ticket, CTAs
+// done) of one launch; launches take slots in turn, and each launch's last CTA
+// zeroes its slot, so launches in flight at the same time (up to kQueueSlots)
+// never share counters.  Zero at load time.
+constexpr int kQueueSlots = 1024;
+__device__ unsigned g_prefill_queue[2 * kQueueSlots];
+
 namespace {
 
 constexpr int kBM = 128;          // query rows per tile (two tiles per CTA)
@@ -99,6 +112,8 @@ struct PrefillParams {
   void* o;
   float* lse;
   unsigned* status;
+  unsigned* next_item;   // work queue: tickets handed out after the first gridDim.x items
+  unsigned* done_ctas;   // the last CTA to finish resets both counters for the next launch
   int B, N, Hq, Hkv, G, n_qblocks, n_ktiles, n_items;   // N: queries per sequence (Nq)
   float scale_log2;
   int causal, o_bf16;
@@ -163,6 +178,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // work item of the CTA's it-th item, published by the producer before that item's
+  // Q copies complete B_QFULL phase it; -1 = no more work
+  volatile int* item_slot = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -201,11 +219,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t once = policy_evict_first();
       int g = 0, it = 0, q_loaded = 0;              // K/V tiles loaded, items started, Q loads issued
       int last_g[2] = {-1, -1};
-      bool ok = true;
-      for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x, ++it) {
+      bool ok = true, clean_end = false;
+      for (int w = blockIdx.x;; ++it) {
+        // Q of the previous item no longer read (this also means its copy landed)
+        if (it > 0 && !wait_or_abort(&bars[B_QEMPTY], (it - 1) & 1, abort_flag, p.status)) break;
+        if (w >= p.n_items) {
+          // no more work: complete B_QFULL phase `it` without a copy
+          item_slot[it & 1] = -1;
+          mbar_arrive(&bars[B_QFULL]);
+          clean_end = true;
+          break;
+        }
+        item_slot[it & 1] = w;
         const Item itm = item_of<KV>(w, p);
         const int kvh = itm.h / p.G;
-        if (it > 0 && !wait_or_abort(&bars[B_QEMPTY], (it - 1) & 1, abort_flag, p.status)) break;
+        const int w_next = (int)gridDim.x + (int)atomicAdd(p.next_item, 1u);
         mbar_arrive_expect_tx(&bars[B_QFULL], 2 * C::kTileBytes);
         ++q_loaded;
 #pragma unroll
@@ -214,8 +242,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int hh = 0; hh < C::kHalves; ++hh)
             tma_load_4d(smem + C::kQOff + t * C::kTileBytes + hh * C::kHalfBytes, &tmQ, &bars[B_QFULL], hh * 64,
                         itm.h, (2 * itm.qb + t) * kBM, itm.b, once);
-        if (w + (int)gridDim.x < p.n_items) {       // warm L2 with the next item's Q
-          const Item nx = item_of<KV>(w + gridDim.x, p);
+        if (w_next < p.n_items) {                   // warm L2 with the next item's Q
+          const Item nx = item_of<KV>(w_next, p);
 #pragma unroll
           for (int t = 0; t < 2; ++t)
 #pragma unroll
@@ -275,9 +303,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
+        if (!ok) break;
+        w = w_next;
       }
-      // no copy may still be landing in shared memory when the CTA exits
-      if (q_loaded > 0) mbar_wait(&bars[B_QFULL], (q_loaded - 1) & 1);
+      // no copy may still be landing in shared memory when the CTA exits (after a clean
+      // end, the wait on B_QEMPTY above already covered the last Q copy)
+      if (!clean_end && q_loaded > 0) mbar_wait(&bars[B_QFULL], (q_loaded - 1) & 1);
       for (int st = 0; st < 2; ++st) {
         if (last_g[st] < 0) continue;
         mbar_wait(&bars[B_KFULL + st], (last_g[st] >> 1) & 1);
@@ -309,11 +340,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       int g = 0, it = 0;                     // K/V tiles consumed, items done
       int pcnt[2] = {0, 0};                  // P_FULL phases consumed per tile
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x, ++it) {
+      for (;; ++it) {
+        if (!wait_or_abort(&bars[B_QFULL], it & 1, abort_flag, p.status)) break;
+        const int w = item_slot[it & 1];
+        if (w < 0) break;                    // no more work
         const Item itm = item_of<KV>(w, p);
         const int g0 = g;
-        ok = wait_or_abort(&bars[B_QFULL], it & 1, abort_flag, p.status) &&
-             wait_or_abort(&bars[B_KFULL + (g0 & 1)], (g0 >> 1) & 1, abort_flag, p.status);
+        ok = wait_or_abort(&bars[B_KFULL + (g0 & 1)], (g0 >> 1) & 1, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
         issue_s(0, g0 & 1);
@@ -365,7 +398,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     int scnt = 0, it = 0;                               // S_FULL phases consumed, items done
     int g_base = 0;                                     // K/V tiles of the previous items
     bool ok = true;
-    for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x, ++it) {
+    for (;; ++it) {
+    if (!wait_or_abort(&bars[B_QFULL], it & 1, abort_flag, p.status)) { ok = false; break; }
+    const int w = item_slot[it & 1];
+    if (w < 0) break;                                   // no more work
     const Item itm = item_of<KV>(w, p);
     const int q_row = (2 * itm.qb + t) * kBM + row;
     const int nkv = t ? itm.n_load : itm.n_kv0;
@@ -522,6 +558,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }
+  if (threadIdx.x == 0 && atomicAdd(p.done_ctas, 1u) == gridDim.x - 1) {
+    // every CTA has taken its last ticket: leave the queue at zero for the next launch
+    atomicExch(p.next_item, 0u);
+    atomicExch(p.done_ctas, 0u);
+  }
+}
+
+// This launch's pair of queue counters on the current device.
+cudaError_t queue_slot(unsigned** next, unsigned** done) {
+  constexpr int kMaxDevices = 64;
+  static void* base[kMaxDevices] = {};
+  static std::atomic<unsigned> launches[kMaxDevices];
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  {
+    std::lock_guard<std::mutex> g(mu);
+    if (!base[dev] && (e = cudaGetSymbolAddress(&base[dev], g_prefill_queue)) != cudaSuccess) return e;
+  }
+  const unsigned slot = launches[dev].fetch_add(1u) % kQueueSlots;
+  *next = static_cast<unsigned*>(base[dev]) + slot;
+  *done = static_cast<unsigned*>(base[dev]) + kQueueSlots + slot;
+  return cudaSuccess;
 }
 
 template <int D, int KV>
@@ -570,6 +631,8 @@ cudaError_t run_prefill(const PrefillLaunch& a, cudaStream_t stream) {
   p.max_blocks = a.max_blocks;
   p.num_blocks = a.num_blocks;
   p.max_keys = KV == KV_PAGED ? a.max_blocks * kPageTokens : (KV == KV_CACHE ? a.capacity : a.N);
+  cudaError_t qe = queue_slot(&p.next_item, &p.done_ctas);
+  if (qe != cudaSuccess) return qe;
   auto kern = prefill_kernel<D, KV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
