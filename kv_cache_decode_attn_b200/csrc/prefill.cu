@@ -82,7 +82,9 @@ struct PrefillCfg {
   static constexpr int kKOff = kQOff + 2 * kTileBytes;    // K stages 0, 1
   static constexpr int kVOff = kKOff + 2 * kTileBytes;    // V stages 0, 1
   static constexpr int kBarOff = kVOff + 2 * kTileBytes;
-  static constexpr int kUsed = kBarOff + 256;
+  static constexpr int kOrderOff = kBarOff + 256;        // cached forms: sequences by length, longest first
+  static constexpr int kMaxOrdered = 256;
+  static constexpr int kUsed = kOrderOff + kMaxOrdered * 4;
   // one CTA per SM: it owns all 512 TMEM columns
   static constexpr int kSmemBytes = (kUsed + 1024) > 120 * 1024 ? (kUsed + 1024) : 120 * 1024;
   static constexpr int kTmemCols = 512;
@@ -139,16 +141,31 @@ struct Item {
   bool bad;                      // invalid length (cached forms): the rows are written as NaN
 };
 
-// Work item w: heaviest causal query blocks first, then consecutive heads (the
-// query heads of one K/V head are adjacent, so its K/V tiles are reused from L2).
+// Work item w.  Dense: heaviest causal query blocks first, then consecutive heads
+// (the query heads of one K/V head are adjacent, so its K/V tiles are reused from
+// L2).  Cached forms, where sequences differ in length: sequences longest first
+// (`order`, or index order when the batch is too large to rank), then K/V head,
+// then query blocks heaviest first, then the heads of that K/V head -- roughly
+// longest-processing-time first, and every reader of one K/V range runs at
+// about the same time, so that range is read from L2.
 template <int KV>
-__device__ __forceinline__ Item item_of(int w, const PrefillParams& p) {
+__device__ __forceinline__ Item item_of(int w, const PrefillParams& p, const int* order) {
   Item it;
-  const int per = p.Hq * p.B;
-  it.qb = p.n_qblocks - 1 - w / per;
-  const int r = w - (w / per) * per;
-  it.h = r % p.Hq;
-  it.b = r / p.Hq;
+  if constexpr (KV == KV_DENSE) {
+    const int per = p.Hq * p.B;
+    it.qb = p.n_qblocks - 1 - w / per;
+    const int r = w - (w / per) * per;
+    it.h = r % p.Hq;
+    it.b = r / p.Hq;
+  } else {
+    const int per_g = p.n_qblocks * p.G;        // items of one (sequence, K/V head)
+    const int per_b = p.Hkv * per_g;
+    const int r = w / per_b, rem = w - r * per_b;
+    it.b = order ? order[r] : r;
+    const int kvh = rem / per_g, rem2 = rem - kvh * per_g;
+    it.qb = p.n_qblocks - 1 - rem2 / p.G;
+    it.h = kvh * p.G + rem2 % p.G;
+  }
   if constexpr (KV == KV_DENSE) {
     it.L = p.N;
     it.off = 0;
@@ -181,6 +198,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   // work item of the CTA's it-th item, published by the producer before that item's
   // Q copies complete B_QFULL phase it; -1 = no more work
   volatile int* item_slot = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  int* order_smem = reinterpret_cast<int*>(smem + C::kOrderOff);
+  const int* order = (KV != KV_DENSE && p.B <= C::kMaxOrdered) ? order_smem : nullptr;
+  if (order) {
+    // rank of each sequence by length, longest first (ties by index)
+    for (int bb = threadIdx.x; bb < p.B; bb += blockDim.x) {
+      const int lb = __ldg(p.seqlens + bb);
+      int rank = 0;
+      for (int o = 0; o < p.B; ++o) {
+        const int lo = __ldg(p.seqlens + o);
+        rank += (lo > lb) || (lo == lb && o < bb);
+      }
+      order_smem[rank] = bb;
+    }
+  }
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -231,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         item_slot[it & 1] = w;
-        const Item itm = item_of<KV>(w, p);
+        const Item itm = item_of<KV>(w, p, order);
         const int kvh = itm.h / p.G;
         const int w_next = (int)gridDim.x + (int)atomicAdd(p.next_item, 1u);
         mbar_arrive_expect_tx(&bars[B_QFULL], 2 * C::kTileBytes);
@@ -243,12 +274,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_4d(smem + C::kQOff + t * C::kTileBytes + hh * C::kHalfBytes, &tmQ, &bars[B_QFULL], hh * 64,
                         itm.h, (2 * itm.qb + t) * kBM, itm.b, once);
         if (w_next < p.n_items) {                   // warm L2 with the next item's Q
-          const Item nx = item_of<KV>(w_next, p);
+          const Item nx = item_of<KV>(w_next, p, order);
 #pragma unroll
           for (int t = 0; t < 2; ++t)
 #pragma unroll
             for (int hh = 0; hh < C::kHalves; ++hh) tma_prefetch_4d(&tmQ, hh * 64, nx.h, (2 * nx.qb + t) * kBM, nx.b);
         }
+        // paged: the physical blocks of tile t, read one tile ahead (the page-table
+        // latency then overlaps the wait for a free stage instead of delaying the copy)
+        constexpr int kBlocks = kBN / kPageTokens;
+        int ids[kBlocks];
+        int nb = 0;
+        auto read_ids = [&](int t) {
+          nb = min(kBlocks, (itm.L - t * kBN + kPageTokens - 1) / kPageTokens);
+          const int32_t* tab = p.page_table + (size_t)itm.b * p.max_blocks + t * kBlocks;
+#pragma unroll
+          for (int jb = 0; jb < kBlocks; ++jb) ids[jb] = jb < nb ? __ldg(tab + jb) : 0;
+        };
+        if constexpr (KV == KV_PAGED) read_ids(0);
         for (int t = 0; t < itm.n_load; ++t, ++g) {
           const int st = g & 1;
           if (g >= 2 && !wait_or_abort(&bars[B_KVEMPTY + st], ((g >> 1) - 1) & 1, abort_flag, p.status)) {
@@ -269,18 +312,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                           hh * 64, kvh, t * kBN, itm.b, keep);
           } else {
             // one 16-row box per physical block holding keys of this tile below L
-            constexpr int kBlocks = kBN / kPageTokens;
-            const int nb = min(kBlocks, (itm.L - t * kBN + kPageTokens - 1) / kPageTokens);
-            const int32_t* tab = p.page_table + (size_t)itm.b * p.max_blocks + t * kBlocks;
-            int ids[kBlocks];
 #pragma unroll
             for (int jb = 0; jb < kBlocks; ++jb) {
-              int id = jb < nb ? __ldg(tab + jb) : 0;
-              if (id < 0 || id >= p.num_blocks) {
+              if (jb < nb && (ids[jb] < 0 || ids[jb] >= p.num_blocks)) {
                 atomicOr(p.status, DEV_PAGE_ID);
-                id = 0;   // keep the byte count; the result is flagged invalid
+                ids[jb] = 0;   // keep the byte count; the result is flagged invalid
               }
-              ids[jb] = id;
             }
             const uint32_t bytes = nb * C::kHalves * kPageTokens * 128;
             mbar_arrive_expect_tx(&bars[B_KFULL + st], bytes);
@@ -301,6 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_load_3d(smem + C::kVOff + st * C::kTileBytes + hh * C::kHalfBytes + jb * kPageTokens * 128, &tmV,
                             &bars[B_VFULL + st], hh * 64, kvh, ids[jb] * kPageTokens, keep);
             }
+            if (t + 1 < itm.n_load) read_ids(t + 1);
           }
         }
         if (!ok) break;
@@ -344,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wait_or_abort(&bars[B_QFULL], it & 1, abort_flag, p.status)) break;
         const int w = item_slot[it & 1];
         if (w < 0) break;                    // no more work
-        const Item itm = item_of<KV>(w, p);
+        const Item itm = item_of<KV>(w, p, order);
         const int g0 = g;
         ok = wait_or_abort(&bars[B_KFULL + (g0 & 1)], (g0 >> 1) & 1, abort_flag, p.status);
         if (!ok) break;
@@ -402,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!wait_or_abort(&bars[B_QFULL], it & 1, abort_flag, p.status)) { ok = false; break; }
     const int w = item_slot[it & 1];
     if (w < 0) break;                                   // no more work
-    const Item itm = item_of<KV>(w, p);
+    const Item itm = item_of<KV>(w, p, order);
     const int q_row = (2 * itm.qb + t) * kBM + row;
     const int nkv = t ? itm.n_load : itm.n_kv0;
     const int g_item = g_base;
