@@ -126,9 +126,10 @@ ATTN_API int attn_prefill_cache(const void* q, const void* k_cache, const void* 
                                 int causal, void* stream);
 
 /*
- * attn_decode_workspace_bytes -- bytes of device workspace attn_decode needs
- * for these sizes (the per-chunk partial outputs and log-sum-exps of the split
- * along the keys).  num_splits as for attn_decode.  Returns 0 for invalid sizes.
+ * attn_decode_workspace_bytes -- bytes of device workspace attn_decode and
+ * attn_decode_fp8 need for these sizes (the per-chunk partial outputs and
+ * log-sum-exps of the split along the keys; the larger of the two, whose key
+ * chunking differs).  num_splits as for attn_decode.  Returns 0 for invalid sizes.
  */
 ATTN_API size_t attn_decode_workspace_bytes(int B, int T, int Hq, int Hkv, int d, int max_seqlen_k, int num_splits);
 

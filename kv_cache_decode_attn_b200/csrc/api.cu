@@ -84,12 +84,13 @@ struct DecodeLayout {
   size_t o_bytes, lse_offset, total;
 };
 
-bool decode_layout(int B, int T, int Hq, int Hkv, int d, int max_seqlen_k, int num_splits, DecodeLayout* out) {
+bool decode_layout(int B, int T, int Hq, int Hkv, int d, int max_seqlen_k, int num_splits, bool fp8,
+                   DecodeLayout* out) {
   if (B < 1 || T < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || max_seqlen_k < 1 || num_splits < 0) return false;
   if (d != 64 && d != 128) return false;
   DecodeLayout L;
   L.R = (Hq / Hkv) * T;
-  L.chunk = decode_chunk_tokens(B, T, Hq / Hkv, Hkv, max_seqlen_k, num_splits);
+  L.chunk = decode_chunk_tokens(B, T, Hq / Hkv, Hkv, max_seqlen_k, num_splits, fp8);
   L.max_chunks = (max_seqlen_k + L.chunk - 1) / L.chunk;
   const size_t items = (size_t)B * Hkv * L.max_chunks;
   L.o_bytes = items * L.R * d * sizeof(float);
@@ -149,9 +150,11 @@ int attn_get_device_status(int clear) {
 }
 
 size_t attn_decode_workspace_bytes(int B, int T, int Hq, int Hkv, int d, int max_seqlen_k, int num_splits) {
-  DecodeLayout L;
-  if (!decode_layout(B, T, Hq, Hkv, d, max_seqlen_k, num_splits, &L)) return 0;
-  return L.total;
+  // enough for attn_decode and for attn_decode_fp8 with the same arguments (their chunking differs)
+  DecodeLayout L, L8;
+  if (!decode_layout(B, T, Hq, Hkv, d, max_seqlen_k, num_splits, false, &L)) return 0;
+  if (!decode_layout(B, T, Hq, Hkv, d, max_seqlen_k, num_splits, true, &L8)) return 0;
+  return L.total > L8.total ? L.total : L8.total;
 }
 
 int attn_prefill(const void* q, const void* k, const void* v, void* o, int o_dtype, float* lse, int B, int Hq,
@@ -216,7 +219,7 @@ int decode_impl(const void* q, const void* k_cache, const void* v_cache, const f
   if (fp8 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
   DecodeLayout L;
-  if (!decode_layout(B, T, Hq, Hkv, d, max_seqlen_k, num_splits, &L)) return ATTN_ERR_INVALID_ARG;
+  if (!decode_layout(B, T, Hq, Hkv, d, max_seqlen_k, num_splits, fp8, &L)) return ATTN_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < L.total || !aligned16(workspace)) return ATTN_ERR_WORKSPACE;
   unsigned* st = status_ptr();
   if (!st) return ATTN_ERR_CUDA;

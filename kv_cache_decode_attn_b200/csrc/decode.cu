@@ -551,19 +551,25 @@ cudaError_t run_split(const CUtensorMap& tk, const CUtensorMap& tv, const SplitP
 
 }  // namespace
 
-int decode_chunk_tokens(int B, int T, int G, int Hkv, int max_seqlen, int num_splits) {
+int decode_chunk_tokens(int B, int T, int G, int Hkv, int max_seqlen, int num_splits, bool fp8) {
   int chunk;
   if (num_splits > 0) {
     chunk = (max_seqlen + num_splits - 1) / num_splits;
   } else {
-    // Long chunks stream longer and leave fewer partials to merge; measured on
-    // B200 the best were 2048 tokens for 16 x 8 sequence-heads up to 32K keys and
-    // 4096 for 8 x 8 up to 128K.  Start at 4096 and halve until the grid holds
-    // about 14 work items per SM (counted as if every sequence had max_seqlen;
-    // row tiles of many new tokens count as separate items).
+    // Long chunks stream longer and leave fewer partials to merge; short ones
+    // balance the grid.  Measured on B200: the warp-MMA kernel (2 CTAs per SM)
+    // was best at 2048 tokens for 16 x 8 sequence-heads up to 32K keys and 4096
+    // for 8 x 8 up to 128K, i.e. about 14 work items per SM; the FP8 kernel for
+    // up to 8 rows (3 CTAs per SM) wants about 21; the tensor-core kernel (1 CTA
+    // per SM, a costly start) wants few long items, about 4 per SM.  Start long
+    // and halve until the grid holds that many items (counted as if every
+    // sequence had max_seqlen; row tiles of many new tokens count separately).
+    const int R = G * T;
+    const bool tc = R > kDecodeMmaRows;
     const long long units = (long long)B * Hkv * decode_row_tiles(T, G);
-    chunk = 4096;
-    while (chunk > 256 && units * ((max_seqlen + chunk - 1) / chunk) < 2048) chunk >>= 1;
+    const long long target = tc ? 640 : (fp8 && R <= 8 ? 3072 : 2048);
+    chunk = tc ? 16384 : 4096;
+    while (chunk > 256 && units * ((max_seqlen + chunk - 1) / chunk) < target) chunk >>= 1;
   }
   // a multiple of both kernels' tiles
   chunk = ((chunk + kDecodeTcTile - 1) / kDecodeTcTile) * kDecodeTcTile;

@@ -42,15 +42,17 @@ constexpr int kTok = 128;    // keys per K/V tile
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
+constexpr int kStages = 3;    // K/V ring stages (S is double-buffered in TMEM)
+
 template <int D>
 struct TcCfg {
   static constexpr int kHalves = D / 64;
   static constexpr int kHalfBytes = kTok * 128;              // 128 rows x 128 B
   static constexpr int kTileBytes = kTok * D * 2;            // one K or V tile (= the Q tile)
   static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + kTileBytes;           // K stages 0, 1
-  static constexpr int kVOff = kKOff + 2 * kTileBytes;       // V stages 0, 1
-  static constexpr int kBarOff = kVOff + 2 * kTileBytes;
+  static constexpr int kKOff = kQOff + kTileBytes;           // K stages
+  static constexpr int kVOff = kKOff + kStages * kTileBytes; // V stages
+  static constexpr int kBarOff = kVOff + kStages * kTileBytes;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;
   static constexpr int kTmemCols = 512;                      // S0 | S1 | O (+ unused)
   static constexpr int kOCol = 256;
@@ -63,8 +65,20 @@ struct TcCfg {
 // O_DONE completes once per PV and is waited on only one tile behind (before a
 // rescale, where PV_{j-2} is known to be done); the epilogue, which may be two
 // PVs behind, waits on O_FINAL, committed once after the last PV.
-enum TcBar { T_Q = 0, T_KFULL = 1, T_VFULL = 3, T_KEMPTY = 5, T_VEMPTY = 7, T_SFULL = 9, T_PFULL = 11, T_ODONE = 13,
-             T_OFINAL = 14, T_DRAIN = 15, T_COUNT = 16 };
+// K/V barriers: one per ring stage; S_FULL / P_FULL: one per S buffer.
+enum TcBar {
+  T_Q = 0,
+  T_KFULL = 1,
+  T_VFULL = T_KFULL + kStages,
+  T_KEMPTY = T_VFULL + kStages,
+  T_VEMPTY = T_KEMPTY + kStages,
+  T_SFULL = T_VEMPTY + kStages,
+  T_PFULL = T_SFULL + 2,
+  T_ODONE = T_PFULL + 2,
+  T_OFINAL,
+  T_DRAIN,
+  T_COUNT
+};
 
 struct TcParams {
   const int32_t* seqlens;
@@ -126,11 +140,13 @@ __global__ void __launch_bounds__(192, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[T_Q], 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars[T_KFULL + s], 1);
       mbar_init(&bars[T_VFULL + s], 1);
       mbar_init(&bars[T_KEMPTY + s], 1);
       mbar_init(&bars[T_VEMPTY + s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[T_SFULL + s], 1);
       mbar_init(&bars[T_PFULL + s], active_warps);
     }
@@ -173,7 +189,9 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
       for (int hh = 0; hh < C::kHalves; ++hh)
         tma_load_4d(smem + C::kQOff + hh * C::kHalfBytes, &tmQ, &bars[T_Q], hh * 64, g * p.G, t0, b, pol);
-      int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};
+      int last_k[kStages], last_v[kStages];
+#pragma unroll
+      for (int s = 0; s < kStages; ++s) last_k[s] = last_v[s] = -1;
       constexpr int kBlocks = kTok / kPageTokens;
       // physical blocks of one tile, read together (the copies' memory clobbers
       // would otherwise serialise one table read per block)
@@ -191,7 +209,7 @@ __global__ void __launch_bounds__(192, 1)
           }
         return nb;
       };
-      // one tensor (K or V) of tile i into ring stage i & 1
+      // one tensor (K or V) of tile i into ring stage i % kStages
       auto load = [&](const CUtensorMap* map, uint8_t* base, uint64_t* full, int i, const int (&ids)[kBlocks],
                       int nb) {
         const int t0 = tok_begin + i * kTok;
@@ -215,20 +233,20 @@ __global__ void __launch_bounds__(192, 1)
       int ids[kBlocks] = {0, 0, 0, 0, 0, 0, 0, 0};
       int nb = PAGED ? read_ids(0, ids) : 0;
       for (int i = 0; i < n_tiles; ++i) {
-        const int st = i & 1;
-        if (i >= 2 && !tc_wait(&bars[T_KEMPTY + st], ((i >> 1) - 1) & 1, abort_flag, p.status)) break;
-        last_k[st] = i;
-        load(&tmK, smem + C::kKOff + st * C::kTileBytes, &bars[T_KFULL + st], i, ids, nb);
-        if (i >= 2 && !tc_wait(&bars[T_VEMPTY + st], ((i >> 1) - 1) & 1, abort_flag, p.status)) break;
-        last_v[st] = i;
-        load(&tmV, smem + C::kVOff + st * C::kTileBytes, &bars[T_VFULL + st], i, ids, nb);
+        const int ks = i % kStages, reuse_ph = ((i / kStages) - 1) & 1;
+        if (i >= kStages && !tc_wait(&bars[T_KEMPTY + ks], reuse_ph, abort_flag, p.status)) break;
+        last_k[ks] = i;
+        load(&tmK, smem + C::kKOff + ks * C::kTileBytes, &bars[T_KFULL + ks], i, ids, nb);
+        if (i >= kStages && !tc_wait(&bars[T_VEMPTY + ks], reuse_ph, abort_flag, p.status)) break;
+        last_v[ks] = i;
+        load(&tmV, smem + C::kVOff + ks * C::kTileBytes, &bars[T_VFULL + ks], i, ids, nb);
         if (PAGED && i + 1 < n_tiles) nb = read_ids(i + 1, ids);
       }
       // no copy may still be landing in shared memory when the CTA exits
       mbar_wait(&bars[T_Q], 0);
-      for (int st = 0; st < 2; ++st) {
-        if (last_k[st] >= 0) mbar_wait(&bars[T_KFULL + st], (last_k[st] >> 1) & 1);
-        if (last_v[st] >= 0) mbar_wait(&bars[T_VFULL + st], (last_v[st] >> 1) & 1);
+      for (int ks = 0; ks < kStages; ++ks) {
+        if (last_k[ks] >= 0) mbar_wait(&bars[T_KFULL + ks], (last_k[ks] / kStages) & 1);
+        if (last_v[ks] >= 0) mbar_wait(&bars[T_VFULL + ks], (last_v[ks] / kStages) & 1);
       }
     }
   } else if (warp == 5) {
@@ -238,15 +256,15 @@ __global__ void __launch_bounds__(192, 1)
       constexpr uint32_t idO = idesc_bf16(kRows, D, 0, 1);
       const uint32_t q_s = smem_u32(smem + C::kQOff);
       auto issue_s = [&](int i) {
-        const int st = i & 1;
-        const uint32_t k_s = smem_u32(smem + C::kKOff + st * C::kTileBytes);
+        const int sb = i & 1, ks = i % kStages;   // S buffer, K/V ring stage
+        const uint32_t k_s = smem_u32(smem + C::kKOff + ks * C::kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
-          tc_mma_ss(tmem + st * 128, smem_desc(q_s + off, 16, 1024), smem_desc(k_s + off, 16, 1024), idS, kk > 0);
+          tc_mma_ss(tmem + sb * 128, smem_desc(q_s + off, 16, 1024), smem_desc(k_s + off, 16, 1024), idS, kk > 0);
         }
-        tc_commit(&bars[T_SFULL + st]);
-        tc_commit(&bars[T_KEMPTY + st]);     // K_i is read only by S_i
+        tc_commit(&bars[T_SFULL + sb]);
+        tc_commit(&bars[T_KEMPTY + ks]);     // K_i is read only by S_i
       };
       bool ok = tc_wait(&bars[T_Q], 0, abort_flag, p.status) &&
                 tc_wait(&bars[T_KFULL], 0, abort_flag, p.status);
@@ -255,24 +273,24 @@ __global__ void __launch_bounds__(192, 1)
         issue_s(0);
       }
       for (int i = 0; ok && i < n_tiles; ++i) {
-        const int st = i & 1;
+        const int sb = i & 1, ks = i % kStages;
         if (i + 1 < n_tiles) {
-          ok = tc_wait(&bars[T_KFULL + ((i + 1) & 1)], ((i + 1) >> 1) & 1, abort_flag, p.status);
+          ok = tc_wait(&bars[T_KFULL + (i + 1) % kStages], ((i + 1) / kStages) & 1, abort_flag, p.status);
           if (!ok) break;
           tc_fence_after();
           issue_s(i + 1);   // its S buffer last held P_{i-1}, whose PV was issued before
         }
-        ok = tc_wait(&bars[T_PFULL + st], (i >> 1) & 1, abort_flag, p.status) &&
-             tc_wait(&bars[T_VFULL + st], (i >> 1) & 1, abort_flag, p.status);
+        ok = tc_wait(&bars[T_PFULL + sb], (i >> 1) & 1, abort_flag, p.status) &&
+             tc_wait(&bars[T_VFULL + ks], (i / kStages) & 1, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t v_s = smem_u32(smem + C::kVOff + st * C::kTileBytes);
+        const uint32_t v_s = smem_u32(smem + C::kVOff + ks * C::kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < kTok / 16; ++kk)
-          tc_mma_ts(tmem + C::kOCol, tmem + st * 128 + kk * 8, smem_desc(v_s + kk * 16 * 128, C::kHalfBytes, 1024),
+          tc_mma_ts(tmem + C::kOCol, tmem + sb * 128 + kk * 8, smem_desc(v_s + kk * 16 * 128, C::kHalfBytes, 1024),
                     idO, (i > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&bars[T_ODONE]);
-        tc_commit(&bars[T_VEMPTY + st]);
+        tc_commit(&bars[T_VEMPTY + ks]);
       }
       // also on a failed wait, so that the epilogue does not wait in vain (abort_flag marks the result)
       tc_commit(&bars[T_OFINAL]);
@@ -359,8 +377,9 @@ __global__ void __launch_bounds__(192, 1)
       // otherwise multiply by p = 0
       const int valid = tok_end - key0;
       if (valid < kTok && warp == 0) {
-        if (!tc_wait(&bars[T_VFULL + st], (i >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-        uint8_t* vst = smem + C::kVOff + st * C::kTileBytes;
+        const int ks = i % kStages;
+        if (!tc_wait(&bars[T_VFULL + ks], (i / kStages) & 1, abort_flag, p.status)) { ok = false; break; }
+        uint8_t* vst = smem + C::kVOff + ks * C::kTileBytes;
         for (int idx = max(valid, 0) * 8 + lane; idx < kTok * 8; idx += 32)
 #pragma unroll
           for (int hh = 0; hh < C::kHalves; ++hh)

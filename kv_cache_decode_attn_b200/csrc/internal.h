@@ -72,7 +72,8 @@ struct AppendLaunch {
 };
 
 // Tokens per split for attn_decode (host heuristic, deterministic in its inputs).
-int decode_chunk_tokens(int B, int T, int G, int Hkv, int max_seqlen, int num_splits);
+// fp8: the call reads an FP8 cache (its kernels want other chunk lengths).
+int decode_chunk_tokens(int B, int T, int G, int Hkv, int max_seqlen, int num_splits, bool fp8);
 
 // Tokens per row tile of the tensor-core decode kernel (G query heads per KV head):
 // as many whole tokens as fit in 128 rows, at most T.
