@@ -53,6 +53,8 @@ WORKLOAD_SETS = {
     # through attn_prefill_cache (the prefill kernel) or attn_decode (split-KV, row-tiled)
     "llama8b_prefill_cache": ("prefill_llama8b", "prefill_chunk_paged"),
     "llama8b_chunked_prefill": ("prefill_llama8b", "prefill_chunk_paged"),
+    # eight new tokens per decode step: the tensor-core split kernel (64 rows per KV head)
+    "llama8b_paged_t8": ("prefill_llama8b", "decode_paged_t8"),
 }
 PREFILL_CACHE_SETS = {"llama8b_prefill_cache"}   # sets whose attend step is attn_prefill_cache
 DEFAULT_SET = "llama8b_layer"

@@ -94,6 +94,9 @@ WORKLOADS = {
     # cached prefix of 4K..16K tokens (chunked prefill / prefix caching)
     "prefill_chunk_paged": Decode("prefill_chunk_paged", B=4, T=512, Hq=32, Hkv=8, d=128, len_lo=4096,
                                   len_hi=16384, paged=True),
+    # eight new tokens per step (speculative verify): 64 query rows per KV head
+    "decode_paged_t8": Decode("decode_paged_t8", B=8, T=8, Hq=64, Hkv=8, d=128, len_lo=32768,
+                              len_hi=131072, paged=True),
 }
 
 SEEDS = {name: 1000 + i for i, name in enumerate(WORKLOADS)}
