@@ -176,16 +176,15 @@ __global__ void __launch_bounds__(DecodeCfg<D, MT, FP8>::kThreads, DecodeCfg<D, 
 
   // ldmatrix lane roles
   const int lm = lane >> 3, lr = lane & 7;
-  bool aborted = false;
 
   for (int i = 0; i < n_tiles; ++i) {
     const int s = i % C::kStages;
     if (!mbar_wait(&full[s], (i / C::kStages) & 1)) {
       atomicOr(p.status, DEV_TIMEOUT);
-      aborted = true;
+      *reinterpret_cast<volatile int*>(abort_flag) = 1;   // every consumer sees it after the barrier below
       break;
     }
-    if (*reinterpret_cast<volatile int*>(abort_flag)) { aborted = true; break; }
+    if (*reinterpret_cast<volatile int*>(abort_flag)) break;
     const uint32_t kbase = smem_u32(smem + s * C::kStageBytes);
     const uint32_t vbase = kbase + C::kTensorBytes;
     const int tok_base = tok_begin + i * kDecodeTile + wsub * 16;
@@ -361,7 +360,9 @@ __global__ void __launch_bounds__(DecodeCfg<D, MT, FP8>::kThreads, DecodeCfg<D, 
   // -------------------------------------------------- merge the four warps
   // every consumer reached here; the ring is idle (all issued tiles consumed)
   asm volatile("bar.sync 1, %0;" ::"n"(C::kConsumerWarps * 32) : "memory");
-  if (aborted || *reinterpret_cast<volatile int*>(abort_flag)) {
+  // one decision for all consumers: a warp that gave up set the shared flag before the
+  // barrier, so none of them can wait at a later named barrier for one that left
+  if (*reinterpret_cast<volatile int*>(abort_flag)) {
     // a wait gave up: leave the partial as NaN so the result is visibly invalid
     const size_t item = ((size_t)b * p.Hkv + g) * p.max_chunks + c;
     for (int r = threadIdx.x; r < p.R; r += C::kConsumerWarps * 32) p.part_lse[item * p.R + r] = NAN;

@@ -138,16 +138,15 @@ __global__ void __launch_bounds__(Fp8StCfg::kThreads, 3)
 #pragma unroll
   for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  bool aborted = false;
 
   for (int i = 0; i < n_tiles; ++i) {
     const int s = i % C::kStages;
     if (!mbar_wait(&full[s], (i / C::kStages) & 1)) {
       atomicOr(p.status, DEV_TIMEOUT);
-      aborted = true;
+      *reinterpret_cast<volatile int*>(abort_flag) = 1;   // every consumer sees it after the barrier below
       break;
     }
-    if (*reinterpret_cast<volatile int*>(abort_flag)) { aborted = true; break; }
+    if (*reinterpret_cast<volatile int*>(abort_flag)) break;
     const uint32_t kbase = smem_u32(smem + s * C::kStageBytes);
     const uint32_t vbase = kbase + C::kTensorBytes;
     const int tok_base = tok_begin + i * kDecodeTile + wsub * 16;
@@ -248,7 +247,9 @@ __global__ void __launch_bounds__(Fp8StCfg::kThreads, 3)
 
   // -------------------------------------------------- merge the four warps
   asm volatile("bar.sync 1, %0;" ::"n"(C::kConsumerWarps * 32) : "memory");
-  if (aborted || *reinterpret_cast<volatile int*>(abort_flag)) {
+  // one decision for all consumers: a warp that gave up set the shared flag before the
+  // barrier, so none of them can wait at a later named barrier for one that left
+  if (*reinterpret_cast<volatile int*>(abort_flag)) {
     for (int r = threadIdx.x; r < p.R; r += C::kConsumerWarps * 32) p.part_lse[item * p.R + r] = NAN;
     return;
   }
