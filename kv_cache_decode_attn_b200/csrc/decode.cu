@@ -358,6 +358,7 @@ __global__ void __launch_bounds__(DecodeCfg<D, MT, FP8>::kThreads, DecodeCfg<D, 
   }
 
   // -------------------------------------------------- merge the four warps
+  launch_dependents();   // the combine kernel may start launching (it waits for this grid)
   // every consumer reached here; the ring is idle (all issued tiles consumed)
   asm volatile("bar.sync 1, %0;" ::"n"(C::kConsumerWarps * 32) : "memory");
   // one decision for all consumers: a warp that gave up set the shared flag before the
@@ -464,6 +465,7 @@ __global__ void __launch_bounds__(256, 4) decode_combine_kernel(const float* __r
                                                              const float* __restrict__ part_lse,
                                                              const int32_t* __restrict__ seqlens, void* o, int o_bf16,
                                                              float* lse, SplitParams p, int B, int paged) {
+  grid_dependency_wait();   // launched early (programmatic dependent launch): the partials are ready after this
   const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int rows = B * p.T * p.Hq;
@@ -499,7 +501,7 @@ __global__ void __launch_bounds__(256, 4) decode_combine_kernel(const float* __r
     for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
     lse_row = M + logf(z);
     // lanes compute the weights of 32 chunks at a time; every lane then walks
-    // those chunks with several independent loads in flight
+    // those chunks with eight independent loads in flight
     const float* src0 = part_o + (item0 * p.R + r) * D + lane * kPer;
     const size_t cstride = (size_t)p.R * D;     // floats between consecutive chunks of this row
     for (int c0 = 0; c0 < nc; c0 += 32) {
@@ -508,16 +510,16 @@ __global__ void __launch_bounds__(256, 4) decode_combine_kernel(const float* __r
       const float wl = (lc == -INFINITY) ? 0.f : expf(lc - lse_row);
       const int n = min(32, nc - c0);
       int i = 0;
-      for (; i + 4 <= n; i += 4) {
-        float w[4];
-        float4 x[4];
+      for (; i + 8 <= n; i += 8) {
+        float w[8];
+        float4 x[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
           w[u] = __shfl_sync(0xffffffffu, wl, i + u);
           x[u] = load_part<kPer>(src0 + (size_t)(c0 + i + u) * cstride);
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) accumulate<kPer>(acc, w[u], x[u]);
+        for (int u = 0; u < 8; ++u) accumulate<kPer>(acc, w[u], x[u]);
       }
       for (; i < n; ++i) {
         const float w = __shfl_sync(0xffffffffu, wl, i);
@@ -634,14 +636,27 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
   }
   if (e != cudaSuccess) return e;
 
+  // the combine kernel is launched as a programmatic dependent of the split kernel:
+  // it starts launching while the split kernel's last CTAs finish and waits for them
   const int rows_out = a.B * a.T * a.Hq;
-  const int blocks = (rows_out * 32 + 255) / 256;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((rows_out * 32 + 255) / 256);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const int paged_i = paged ? 1 : 0;
   if (a.d == 128)
-    decode_combine_kernel<128><<<blocks, 256, 0, stream>>>(a.part_o, a.part_lse, a.seqlens, a.o, a.o_bf16, a.lse, sp,
-                                                           a.B, paged ? 1 : 0);
+    e = cudaLaunchKernelEx(&cfg, decode_combine_kernel<128>, (const float*)a.part_o, (const float*)a.part_lse,
+                           a.seqlens, a.o, a.o_bf16, a.lse, sp, a.B, paged_i);
   else
-    decode_combine_kernel<64><<<blocks, 256, 0, stream>>>(a.part_o, a.part_lse, a.seqlens, a.o, a.o_bf16, a.lse, sp,
-                                                          a.B, paged ? 1 : 0);
+    e = cudaLaunchKernelEx(&cfg, decode_combine_kernel<64>, (const float*)a.part_o, (const float*)a.part_lse,
+                           a.seqlens, a.o, a.o_bf16, a.lse, sp, a.B, paged_i);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -246,6 +246,7 @@ __global__ void __launch_bounds__(Fp8StCfg::kThreads, 3)
   }
 
   // -------------------------------------------------- merge the four warps
+  launch_dependents();   // the combine kernel may start launching (it waits for this grid)
   asm volatile("bar.sync 1, %0;" ::"n"(C::kConsumerWarps * 32) : "memory");
   // one decision for all consumers: a warp that gave up set the shared flag before the
   // barrier, so none of them can wait at a later named barrier for one that left

@@ -393,6 +393,7 @@ __global__ void __launch_bounds__(192, 1)
     }
 
     // ---------------------------------------------------------- epilogue
+    launch_dependents();   // the combine kernel may start launching (it waits for this grid)
     if (ok && tc_wait(&bars[T_OFINAL], 0, abort_flag, p.status) && !*abort_flag) {
       tc_fence_after();
       float* out = p.part_o + (row0 + row) * D;

@@ -210,6 +210,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Programmatic dependent launch: let the next kernel on the stream start launching
+// (its CTAs still wait in grid_dependency_wait until this grid has finished and
+// its writes are visible), and that wait.
+__device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // max(a, b, c) in one instruction (sm_100)
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
