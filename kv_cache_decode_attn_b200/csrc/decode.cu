@@ -45,6 +45,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 template <int D, int MT, bool FP8>
 struct DecodeCfg {
   static_assert(!FP8 || D == 128, "FP8 caches are built for d = 128");
+  static_assert(MT == 1 || FP8, "bf16 caches with more than 16 rows run on the tensor-core kernel");
   static constexpr int kConsumerWarps = 4 * MT;
   static constexpr int kThreads = 32 * (kConsumerWarps + 1);
   static constexpr int kHalves = (FP8 ? D : 2 * D) / 128;   // 128-byte swizzle spans per token row
@@ -501,7 +502,7 @@ __global__ void __launch_bounds__(256, 4) decode_combine_kernel(const float* __r
     for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
     lse_row = M + logf(z);
     // lanes compute the weights of 32 chunks at a time; every lane then walks
-    // those chunks with eight independent loads in flight
+    // those chunks with four independent loads in flight
     const float* src0 = part_o + (item0 * p.R + r) * D + lane * kPer;
     const size_t cstride = (size_t)p.R * D;     // floats between consecutive chunks of this row
     for (int c0 = 0; c0 < nc; c0 += 32) {
@@ -510,16 +511,16 @@ __global__ void __launch_bounds__(256, 4) decode_combine_kernel(const float* __r
       const float wl = (lc == -INFINITY) ? 0.f : expf(lc - lse_row);
       const int n = min(32, nc - c0);
       int i = 0;
-      for (; i + 8 <= n; i += 8) {
-        float w[8];
-        float4 x[8];
+      for (; i + 4 <= n; i += 4) {
+        float w[4];
+        float4 x[4];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < 4; ++u) {
           w[u] = __shfl_sync(0xffffffffu, wl, i + u);
           x[u] = load_part<kPer>(src0 + (size_t)(c0 + i + u) * cstride);
         }
 #pragma unroll
-        for (int u = 0; u < 8; ++u) accumulate<kPer>(acc, w[u], x[u]);
+        for (int u = 0; u < 4; ++u) accumulate<kPer>(acc, w[u], x[u]);
       }
       for (; i < n; ++i) {
         const float w = __shfl_sync(0xffffffffu, wl, i);
@@ -568,7 +569,7 @@ int decode_chunk_tokens(int B, int T, int G, int Hkv, int max_seqlen, int num_sp
     // and halve until the grid holds that many items (counted as if every
     // sequence had max_seqlen; row tiles of many new tokens count separately).
     const int R = G * T;
-    const bool tc = R > kDecodeMmaRows;
+    const bool tc = decode_uses_tc(R, fp8);
     const long long units = (long long)B * Hkv * decode_row_tiles(T, G);
     const long long target = tc ? 640 : (fp8 && R <= 8 ? 3072 : 2048);
     chunk = tc ? 16384 : 4096;
@@ -607,7 +608,7 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
 
   // K/V viewed as 3-D {d, Hkv, rows}: rows = B * capacity (contiguous) or num_blocks * 16 (paged)
   const uint64_t rows = paged ? (uint64_t)a.num_blocks * kPageTokens : (uint64_t)a.B * a.capacity;
-  const bool tc = R > kDecodeMmaRows;
+  const bool tc = decode_uses_tc(R, a.fp8 != 0);
   const uint32_t box_rows = paged ? kPageTokens : (tc ? kDecodeTcTile : kDecodeTile);
   CUtensorMap tk, tv;
   const int eb = a.fp8 ? 1 : 2;   // bytes per cached element
@@ -619,7 +620,7 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
 
   cudaError_t e;
   if (a.fp8) {
-    // api.cu admits d == 128 and at most kDecodeMmaRows rows per KV head
+    // api.cu admits d == 128 and at most kFp8MaxRows rows per KV head
     if (R <= 8) e = launch_decode_fp8_rows8(tk, tv, sp, a.B, paged, stream);
     else if (R <= 16) e = paged ? run_split<128, 1, true, true>(tk, tv, sp, a.B, stream)
                            : run_split<128, 1, false, true>(tk, tv, sp, a.B, stream);
@@ -627,12 +628,10 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
                    : run_split<128, 2, false, true>(tk, tv, sp, a.B, stream);
   } else if (tc) {
     e = launch_decode_tc(a, tk, tv, stream);
-  } else if (a.d == 128) {
-    if (R <= 16) e = paged ? run_split<128, 1, true>(tk, tv, sp, a.B, stream) : run_split<128, 1, false>(tk, tv, sp, a.B, stream);
-    else e = paged ? run_split<128, 2, true>(tk, tv, sp, a.B, stream) : run_split<128, 2, false>(tk, tv, sp, a.B, stream);
+  } else if (a.d == 128) {   // at most kDecodeMmaRows (16) rows: one row group
+    e = paged ? run_split<128, 1, true>(tk, tv, sp, a.B, stream) : run_split<128, 1, false>(tk, tv, sp, a.B, stream);
   } else {
-    if (R <= 16) e = paged ? run_split<64, 1, true>(tk, tv, sp, a.B, stream) : run_split<64, 1, false>(tk, tv, sp, a.B, stream);
-    else e = paged ? run_split<64, 2, true>(tk, tv, sp, a.B, stream) : run_split<64, 2, false>(tk, tv, sp, a.B, stream);
+    e = paged ? run_split<64, 1, true>(tk, tv, sp, a.B, stream) : run_split<64, 1, false>(tk, tv, sp, a.B, stream);
   }
   if (e != cudaSuccess) return e;
 

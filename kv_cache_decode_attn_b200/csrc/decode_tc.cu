@@ -12,10 +12,12 @@
 // keys up to the last one its last token sees.  Warp roles:
 //   warps 0..3  softmax: thread i owns row i (TMEM lane i); warps whose rows are
 //               all >= R stay idle;
-//   warp 4      TMA producer: Q once, then 128-token K/V tiles (contiguous: one
-//               128-row box per 64 columns of d; paged: one 16-row box per
-//               physical block, its page-table entry checked first) into a
-//               2-stage ring with the evict-first L2 policy;
+//   warps 4, 6  TMA producers: warp 4 loads Q once and the K tiles, warp 6 the V
+//               tiles, each into its own 3-stage ring with the evict-first L2
+//               policy (128-token tiles; contiguous: one 128-row box per 64
+//               columns of d; paged: one 16-row box per physical block, its
+//               page-table entry checked first).  K is released by S_j, V only by
+//               PV_j, so separate producers let the K ring run ahead;
 //   warp 5      MMA issuer: S_j = Q K_j^T (SS) into one of two TMEM S buffers,
 //               O += P_j V_j (P read from TMEM, where the softmax wrote it over
 //               the consumed S columns).  S_{j+1} is issued before PV_j, so the
@@ -103,7 +105,7 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
 }
 
 template <int D, bool PAGED>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(224, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const TcParams p) {
   using C = TcCfg<D>;
@@ -177,28 +179,33 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
-    // ------------------------------------------------------------- TMA producer
+  if (warp == 4 || warp == 6) {
+    // ------------------------------------------------------------- TMA producers
     if (lane == 0) {
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
+      const bool is_k = warp == 4;
+      const CUtensorMap* map = is_k ? &tmK : &tmV;
+      prefetch_tmap(map);
       const uint64_t pol = policy_evict_first();
-      // Q rows (t, head g*G + hh) for t0 <= t < t0 + TT, hh < G: one box {64, G, TT, 1} per half
-      // of d (the full box is counted, also where tokens >= T are zero-filled)
-      mbar_arrive_expect_tx(&bars[T_Q], p.TT * p.G * D * 2);
+      if (is_k) {
+        // Q rows (t, head g*G + hh) for t0 <= t < t0 + TT, hh < G: one box {64, G, TT, 1} per half
+        // of d (the full box is counted, also where tokens >= T are zero-filled)
+        mbar_arrive_expect_tx(&bars[T_Q], p.TT * p.G * D * 2);
 #pragma unroll
-      for (int hh = 0; hh < C::kHalves; ++hh)
-        tma_load_4d(smem + C::kQOff + hh * C::kHalfBytes, &tmQ, &bars[T_Q], hh * 64, g * p.G, t0, b, pol);
-      int last_k[kStages], last_v[kStages];
+        for (int hh = 0; hh < C::kHalves; ++hh)
+          tma_load_4d(smem + C::kQOff + hh * C::kHalfBytes, &tmQ, &bars[T_Q], hh * 64, g * p.G, t0, b, pol);
+      }
+      uint8_t* ring = smem + (is_k ? C::kKOff : C::kVOff);
+      const int full0 = is_k ? T_KFULL : T_VFULL, empty0 = is_k ? T_KEMPTY : T_VEMPTY;
+      int last[kStages];
 #pragma unroll
-      for (int s = 0; s < kStages; ++s) last_k[s] = last_v[s] = -1;
+      for (int s = 0; s < kStages; ++s) last[s] = -1;
       constexpr int kBlocks = kTok / kPageTokens;
       // physical blocks of one tile, read together (the copies' memory clobbers
       // would otherwise serialise one table read per block)
       auto read_ids = [&](int i, int (&ids)[kBlocks]) {
-        const int t0 = tok_begin + i * kTok;
-        const int nb = min(kBlocks, (tok_end - t0 + kPageTokens - 1) / kPageTokens);
-        const int32_t* tab = p.page_table + (size_t)b * p.max_blocks + t0 / kPageTokens;
+        const int tt = tok_begin + i * kTok;
+        const int nb = min(kBlocks, (tok_end - tt + kPageTokens - 1) / kPageTokens);
+        const int32_t* tab = p.page_table + (size_t)b * p.max_blocks + tt / kPageTokens;
 #pragma unroll
         for (int j = 0; j < kBlocks; ++j) ids[j] = j < nb ? __ldg(tab + j) : 0;
 #pragma unroll
@@ -209,15 +216,20 @@ __global__ void __launch_bounds__(192, 1)
           }
         return nb;
       };
-      // one tensor (K or V) of tile i into ring stage i % kStages
-      auto load = [&](const CUtensorMap* map, uint8_t* base, uint64_t* full, int i, const int (&ids)[kBlocks],
-                      int nb) {
-        const int t0 = tok_begin + i * kTok;
+      int ids[kBlocks] = {0, 0, 0, 0, 0, 0, 0, 0};
+      int nb = PAGED ? read_ids(0, ids) : 0;
+      for (int i = 0; i < n_tiles; ++i) {
+        const int ks = i % kStages;
+        if (i >= kStages && !tc_wait(&bars[empty0 + ks], ((i / kStages) - 1) & 1, abort_flag, p.status)) break;
+        last[ks] = i;
+        uint8_t* base = ring + ks * C::kTileBytes;
+        uint64_t* full = &bars[full0 + ks];
+        const int tt = tok_begin + i * kTok;
         if (!PAGED) {
           mbar_arrive_expect_tx(full, C::kTileBytes);
 #pragma unroll
           for (int hh = 0; hh < C::kHalves; ++hh)
-            tma_load_3d(base + hh * C::kHalfBytes, map, full, hh * 64, g, b * p.capacity + t0, pol);
+            tma_load_3d(base + hh * C::kHalfBytes, map, full, hh * 64, g, b * p.capacity + tt, pol);
         } else {
           mbar_arrive_expect_tx(full, nb * C::kHalves * kPageTokens * 128);
 #pragma unroll
@@ -228,26 +240,13 @@ __global__ void __launch_bounds__(192, 1)
               tma_load_3d(base + hh * C::kHalfBytes + j * kPageTokens * 128, map, full, hh * 64, g,
                           ids[j] * kPageTokens, pol);
           }
+          if (i + 1 < n_tiles) nb = read_ids(i + 1, ids);
         }
-      };
-      int ids[kBlocks] = {0, 0, 0, 0, 0, 0, 0, 0};
-      int nb = PAGED ? read_ids(0, ids) : 0;
-      for (int i = 0; i < n_tiles; ++i) {
-        const int ks = i % kStages, reuse_ph = ((i / kStages) - 1) & 1;
-        if (i >= kStages && !tc_wait(&bars[T_KEMPTY + ks], reuse_ph, abort_flag, p.status)) break;
-        last_k[ks] = i;
-        load(&tmK, smem + C::kKOff + ks * C::kTileBytes, &bars[T_KFULL + ks], i, ids, nb);
-        if (i >= kStages && !tc_wait(&bars[T_VEMPTY + ks], reuse_ph, abort_flag, p.status)) break;
-        last_v[ks] = i;
-        load(&tmV, smem + C::kVOff + ks * C::kTileBytes, &bars[T_VFULL + ks], i, ids, nb);
-        if (PAGED && i + 1 < n_tiles) nb = read_ids(i + 1, ids);
       }
       // no copy may still be landing in shared memory when the CTA exits
-      mbar_wait(&bars[T_Q], 0);
-      for (int ks = 0; ks < kStages; ++ks) {
-        if (last_k[ks] >= 0) mbar_wait(&bars[T_KFULL + ks], (last_k[ks] / kStages) & 1);
-        if (last_v[ks] >= 0) mbar_wait(&bars[T_VFULL + ks], (last_v[ks] / kStages) & 1);
-      }
+      if (is_k) mbar_wait(&bars[T_Q], 0);
+      for (int ks = 0; ks < kStages; ++ks)
+        if (last[ks] >= 0) mbar_wait(&bars[full0 + ks], (last[ks] / kStages) & 1);
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------- MMA issuer
@@ -467,7 +466,7 @@ cudaError_t run_tc(const DecodeLaunch& a, const CUtensorMap& tk, const CUtensorM
   if (e != cudaSuccess) return e;
   if ((long long)a.max_chunks * row_tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
   dim3 grid(a.max_chunks * row_tiles, a.Hkv, a.B);
-  kern<<<grid, 192, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  kern<<<grid, 224, C::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 

@@ -11,10 +11,16 @@ namespace kvattn {
 constexpr int kPageTokens = 16;   // tokens per physical KV block
 constexpr int kDecodeTile = 64;   // tokens per pipeline stage of the warp-MMA decode kernel
 constexpr int kDecodeTcTile = 128;  // tokens per K/V tile of the tensor-core decode kernel
-// Above this many query rows per KV head the tensor-core kernel runs.  Up to 32
-// the warp-MMA kernel is faster: its four consumer warps use all four SM
-// sub-partitions, while the tensor-core kernel's rows all sit in one warp.
-constexpr int kDecodeMmaRows = 32;
+// Above this many query rows per KV head the tensor-core kernel runs (bf16
+// caches).  Measured on B200 (paged Llama decode, 8 KV heads x 8 sequences):
+// 32 rows ran at 5.7 TB/s there against 4.5 TB/s on the warp-MMA kernel, whose
+// row groups each re-read the K/V fragments; up to 16 rows the warp-MMA kernel
+// streams at the HBM rate.
+constexpr int kDecodeMmaRows = 16;
+// FP8 caches have warp-MMA kernels only: at most this many rows per KV head.
+constexpr int kFp8MaxRows = 32;
+// Whether attn_decode runs the tensor-core split kernel for R rows per KV head.
+inline bool decode_uses_tc(int R, bool fp8) { return !fp8 && R > kDecodeMmaRows; }
 
 struct DecodeLaunch {
   const void* q;
@@ -78,7 +84,7 @@ int decode_chunk_tokens(int B, int T, int G, int Hkv, int max_seqlen, int num_sp
 // Tokens per row tile of the tensor-core decode kernel (G query heads per KV head):
 // as many whole tokens as fit in 128 rows, at most T.
 inline int decode_tc_tile_tokens(int T, int G) { return T < 128 / G ? T : 128 / G; }
-// Row tiles per KV head: 1 on the warp-MMA path (at most kDecodeMmaRows rows).
+// Row tiles per KV head (1 unless the rows exceed one 128-row tensor-core tile).
 inline int decode_row_tiles(int T, int G) {
   if (G * T <= kDecodeMmaRows) return 1;
   const int tt = decode_tc_tile_tokens(T, G);
