@@ -223,9 +223,21 @@ def append_and_attend(kv, wd, kc, vc, q, k_new, v_new, cache_lens, seqlens, tabl
 def decode_kernel_name(wd, prefill_cache=False) -> str:
     if prefill_cache:
         return "prefill_kernel<128, paged cache>" if wd.paged else "prefill_kernel<128, cache>"
+    return f"{decode_kernel(wd)[0]} + decode_combine_kernel"
+
+
+def decode_kernel(wd):
+    """(name, source files) of the kernel attn_decode picks for this shape: bf16 up
+    to 16 query rows per KV head on warp-level MMAs, more on tcgen05; FP8 up to
+    8 rows on the transposed-product kernel, up to 32 on the split kernel."""
     R = wd.Hq // wd.Hkv * wd.T
-    split = "decode_split_kernel" + ("<fp8>" if wd.fp8 else "") if R <= 32 else "decode_tc_kernel"
-    return f"{split} + decode_combine_kernel"
+    if wd.fp8:
+        if R <= 8:
+            return "decode_fp8_st_kernel", ("decode_fp8.cu", "split.cuh", "decode.cu")
+        return "decode_split_kernel<fp8>", ("decode.cu", "split.cuh")
+    if R <= 16:
+        return "decode_split_kernel", ("decode.cu", "split.cuh")
+    return "decode_tc_kernel", ("decode_tc.cu", "decode.cu")
 
 
 def run_ours(args, world, rank, local):
@@ -326,7 +338,7 @@ def run_ours(args, world, rank, local):
     peaks, peak_src = load_peaks()
     pf_kernel_tflops = flops / (pf_ms / K * 1e-3) / 1e12          # per launch, this rank
     dec_kernel_gbs = dbytes / (dec_ms / K * 1e-3) / 1e9
-    traffic = load_traffic()
+    traffic = load_traffic(args.workload, wd)
     roof_pf = {"bound": "tensor", "achieved": round(pf_kernel_tflops, 1), "peak": peaks["bf16_tflops"],
                "unit": "TFLOP/s", "frac": round(pf_kernel_tflops / peaks["bf16_tflops"], 4),
                "frac_of_sustained": round(pf_kernel_tflops / peaks["bf16_tflops_sustained"], 4),
@@ -340,13 +352,13 @@ def run_ours(args, world, rank, local):
         roof_dec = {"bound": "tensor", "achieved": round(dec_kernel_tflops, 1), "peak": peaks["bf16_tflops"],
                     "unit": "TFLOP/s", "frac": round(dec_kernel_tflops / peaks["bf16_tflops"], 4),
                     "frac_of_sustained": round(dec_kernel_tflops / peaks["bf16_tflops_sustained"], 4),
-                    "peak_source": f"{peak_src} (bf16 burst)", "traffic": None,
+                    "peak_source": f"{peak_src} (bf16 burst)", "traffic": traffic.get("decode"),
                     "kernel": decode_kernel_name(wd, prefill_cache),
                     "flops_per_launch": dflops, "bytes_per_launch": dbytes, "launch_ms": round(dec_ms / K, 4)}
     else:
         roof_dec = {"bound": "hbm", "achieved": round(dec_kernel_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": round(dec_kernel_gbs / peaks["hbm_gbs"], 4), "peak_source": f"{peak_src} (copy)",
-                    "traffic": traffic.get("decode") if not wd.fp8 and wd.T * wd.Hq // wd.Hkv <= 32 else None,
+                    "traffic": traffic.get("decode"),
                     "kernel": decode_kernel_name(wd, prefill_cache), "bytes_per_launch": dbytes,
                     "launch_ms": round(dec_ms / K, 4)}
 
@@ -449,26 +461,43 @@ def run_e2e(kv, torch, dev, stream, wp, wd, q, k, v, case, table, msk, ws, args,
             "decode": {"value": round(dbytes / (dec_max * 1e-3) / 1e9, 1), "unit": "GB/s"}}
 
 
-def load_traffic():
-    """Per-launch DRAM bytes (ncu dram__bytes_read + dram__bytes_write) from the
-    committed profile summary, kept only while the kernel source it was measured
-    on is unchanged (first 16 hex digits of its sha256)."""
+def source_hash(files) -> str:
+    """First 16 hex digits of the sha256 over the named csrc files, in order."""
     import hashlib
+    h = hashlib.sha256()
+    for name in files:
+        with open(os.path.join(ROOT, "kv_cache_decode_attn_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(workload, wd):
+    """Per-launch DRAM bytes (ncu dram__bytes_read.sum + dram__bytes_write.sum,
+    summed over the leg's kernels) from the committed profile summary, for this
+    workload only, and kept only while the kernel sources it was measured on are
+    unchanged."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            d = json.load(f)
-    except (OSError, ValueError):
+            entries = json.load(f)["entries"]
+    except (OSError, ValueError, KeyError):
         return {}
+    prefill_cache = workload in PREFILL_CACHE_SETS
+    want = {"prefill": ("prefill_kernel<128>", ("prefill.cu",)),
+            "decode": ("prefill_kernel<128>", ("prefill.cu",)) if prefill_cache else decode_kernel(wd)}
     out = {}
-    for key, src in (("prefill", "prefill.cu"), ("decode", "decode.cu")):
-        try:
-            with open(os.path.join(ROOT, "kv_cache_decode_attn_b200", "csrc", src), "rb") as f:
-                h = hashlib.sha256(f.read()).hexdigest()[:16]
-        except OSError:
+    for e in entries:
+        leg = e.get("leg")
+        if e.get("workload") != workload or leg not in want:
             continue
-        if d.get(f"{key}_source_sha256_16") == h and key in d:
-            out[key] = d[key]
+        kernel, files = want[leg]
+        try:
+            ok = e.get("kernel") == kernel and tuple(e["sources"]) == tuple(files) \
+                and e.get("sha256_16") == source_hash(files)
+        except (OSError, KeyError):
+            ok = False
+        if ok:
+            out[leg] = e["bytes"]
     return out
 
 
