@@ -484,7 +484,7 @@ def load_traffic(workload, wd):
         return {}
     prefill_cache = workload in PREFILL_CACHE_SETS
     want = {"prefill": ("prefill_kernel<128>", ("prefill.cu",)),
-            "decode": ("prefill_kernel<128>", ("prefill.cu",)) if prefill_cache else decode_kernel(wd)}
+            "decode": (decode_kernel_name(wd, True), ("prefill.cu",)) if prefill_cache else decode_kernel(wd)}
     out = {}
     for e in entries:
         leg = e.get("leg")

@@ -460,73 +460,132 @@ __device__ __forceinline__ void accumulate(float (&acc)[kPer], float w, float4 x
   }
 }
 
-// One warp per output row (b, t, h): merge the chunk partials of that row.
+// Merge the chunk partials of each output row (b, t, h).  wpr warps (1, 2, 4 or 8)
+// share a row: warp w of the row takes chunks w, w + wpr, ...; their weighted sums
+// meet in shared memory.  The sequence length is read before the wait on the split
+// kernel (that kernel does not write it); after the wait every warp issues its first
+// kBatch partial loads together with the row's LSE loads, so a row costs about two
+// dependent memory round trips.
 template <int D>
-__global__ void __launch_bounds__(256, 4) decode_combine_kernel(const float* __restrict__ part_o,
+__global__ void __launch_bounds__(256, 2) decode_combine_kernel(const float* __restrict__ part_o,
                                                              const float* __restrict__ part_lse,
                                                              const int32_t* __restrict__ seqlens, void* o, int o_bf16,
-                                                             float* lse, SplitParams p, int B, int paged) {
-  grid_dependency_wait();   // launched early (programmatic dependent launch): the partials are ready after this
-  const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
+                                                             float* lse, SplitParams p, int B, int paged, int wpr) {
+  constexpr int kPer = D / 32;    // output columns per lane
+  constexpr int kBatch = 8;       // partial loads in flight per lane
+  __shared__ float4 red[8][32];   // one float4 per lane of each of the 8 warps
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wi = warp & (wpr - 1);
+  const int row = (blockIdx.x * 8 + warp) / wpr;
   const int rows = B * p.T * p.Hq;
-  if (warp_global >= rows) return;
-  const int h = warp_global % p.Hq;
-  const int t = (warp_global / p.Hq) % p.T;
-  const int b = warp_global / (p.Hq * p.T);
+  const bool live = row < rows;
+  const int h = row % p.Hq;
+  const int t = (row / p.Hq) % p.T;
+  const int b = row / (p.Hq * p.T);
   const int g = h / p.G, r = t * p.G + (h - g * p.G);
-  constexpr int kPer = D / 32;   // output columns per lane
+  bool bad = true;
+  int nc = 0;
+  if (live) {
+    const int L = seqlens[b];
+    bad = seqlen_bad(L, p.T, p.max_seqlen, paged != 0, p.capacity, p.max_blocks);
+    if (!bad) nc = (L + p.chunk - 1) / p.chunk;
+  }
+  grid_dependency_wait();   // launched early (programmatic dependent launch): the partials are ready after this
+
   float acc[kPer];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
-  float lse_row;
-
-  const int L = seqlens[b];
-  if (seqlen_bad(L, p.T, p.max_seqlen, paged != 0, p.capacity, p.max_blocks)) {
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) acc[e] = NAN;
-    lse_row = NAN;
-  } else {
-    const int nc = (L + p.chunk - 1) / p.chunk;
+  float lse_row = -INFINITY;
+  if (nc > 0) {
     const size_t item0 = ((size_t)b * p.Hkv + g) * p.max_chunks;
-    float M = -INFINITY;
-    for (int c = lane; c < nc; c += 32) M = fmaxf(M, part_lse[(item0 + c) * p.R + r]);
+    const float* lse0 = part_lse + item0 * p.R + r;            // chunk c at lse0[c * R]
+    const float* src0 = part_o + (item0 * p.R + r) * D + lane * kPer;
+    const size_t cstride = (size_t)p.R * D;                    // floats between consecutive chunks of this row
+    const int n0 = min(nc, 32);
+    const float lc0 = lane < n0 ? __ldg(lse0 + (size_t)lane * p.R) : -INFINITY;
+    float4 x[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int c = wi + u * wpr;
+      x[u] = c < n0 ? load_part<kPer>(src0 + (size_t)c * cstride) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    // log-sum-exp over the chunks: every lane keeps a (max, sum) pair, then the pairs merge
+    float m = lc0, sum = lc0 == -INFINITY ? 0.f : 1.f;
+    for (int c = 32 + lane; c < nc; c += 32) {
+      const float lc = __ldg(lse0 + (size_t)c * p.R);
+      if (lc == -INFINITY) continue;
+      if (lc > m) {
+        sum = sum * expf(m - lc) + 1.f;
+        m = lc;
+      } else {
+        sum += expf(lc - m);
+      }
+    }
+    float M = m;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float z = 0.f;
-    for (int c = lane; c < nc; c += 32) {
-      const float lc = part_lse[(item0 + c) * p.R + r];
-      z += (lc == -INFINITY) ? 0.f : expf(lc - M);
-    }
+    float z = m == -INFINITY ? 0.f : sum * expf(m - M);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
     lse_row = M + logf(z);
-    // lanes compute the weights of 32 chunks at a time; every lane then walks
-    // those chunks with four independent loads in flight
-    const float* src0 = part_o + (item0 * p.R + r) * D + lane * kPer;
-    const size_t cstride = (size_t)p.R * D;     // floats between consecutive chunks of this row
-    for (int c0 = 0; c0 < nc; c0 += 32) {
-      const int c = c0 + lane;
-      const float lc = c < nc ? part_lse[(item0 + c) * p.R + r] : -INFINITY;
-      const float wl = (lc == -INFINITY) ? 0.f : expf(lc - lse_row);
-      const int n = min(32, nc - c0);
-      int i = 0;
-      for (; i + 4 <= n; i += 4) {
-        float w[4];
-        float4 x[4];
+    // chunk c of the first 32 has its weight on lane c
+    const float wl0 = lc0 == -INFINITY ? 0.f : expf(lc0 - lse_row);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          w[u] = __shfl_sync(0xffffffffu, wl, i + u);
-          x[u] = load_part<kPer>(src0 + (size_t)(c0 + i + u) * cstride);
+    for (int u = 0; u < kBatch; ++u) {
+      const int c = wi + u * wpr;
+      const float w = __shfl_sync(0xffffffffu, wl0, c & 31);
+      if (c < n0) accumulate<kPer>(acc, w, x[u]);
+    }
+    // what the first batch did not cover: more chunks of the first 32, later groups of 32
+    for (int g0 = 0; g0 < nc; g0 += 32) {
+      const int n = min(32, nc - g0);
+      const int first = g0 == 0 ? wi + kBatch * wpr : wi;
+      if (first >= n) continue;
+      const float lc = g0 == 0 ? lc0 : (lane < n ? __ldg(lse0 + (size_t)(g0 + lane) * p.R) : -INFINITY);
+      const float wl = lc == -INFINITY ? 0.f : expf(lc - lse_row);
+      for (int j0 = first; j0 < n; j0 += kBatch * wpr) {
+        float4 y[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+          const int j = j0 + u * wpr;
+          y[u] = j < n ? load_part<kPer>(src0 + (size_t)(g0 + j) * cstride) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) accumulate<kPer>(acc, w[u], x[u]);
-      }
-      for (; i < n; ++i) {
-        const float w = __shfl_sync(0xffffffffu, wl, i);
-        accumulate<kPer>(acc, w, load_part<kPer>(src0 + (size_t)(c0 + i) * cstride));
+        for (int u = 0; u < kBatch; ++u) {
+          const int j = j0 + u * wpr;
+          const float w = __shfl_sync(0xffffffffu, wl, j & 31);
+          if (j < n) accumulate<kPer>(acc, w, y[u]);
+        }
       }
     }
+  }
+  if (wpr > 1) {   // the row's warps add up in shared memory; its first warp writes
+    if (wi != 0) {
+      float4 v = make_float4(acc[0], acc[1], 0.f, 0.f);
+      if constexpr (kPer == 4) {
+        v.z = acc[2];
+        v.w = acc[3];
+      }
+      red[warp][lane] = v;
+    }
+    __syncthreads();
+    if (wi == 0) {
+      for (int k = 1; k < wpr; ++k) {
+        const float4 v = red[warp + k][lane];
+        acc[0] += v.x;
+        acc[1] += v.y;
+        if constexpr (kPer == 4) {
+          acc[2] += v.z;
+          acc[3] += v.w;
+        }
+      }
+    }
+  }
+  if (!live || wi != 0) return;
+  if (bad) {
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) acc[e] = NAN;
+    lse_row = NAN;
   }
   const size_t orow = (((size_t)b * p.T + t) * p.Hq + h) * D + lane * kPer;
   if (o_bf16) {
@@ -637,9 +696,12 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
 
   // the combine kernel is launched as a programmatic dependent of the split kernel:
   // it starts launching while the split kernel's last CTAs finish and waits for them
-  const int rows_out = a.B * a.T * a.Hq;
+  // warps per output row: enough that each warp merges at most four chunks
+  int wpr = 1;
+  while (wpr < 8 && wpr * 4 < sp.max_chunks) wpr *= 2;
+  const long long rows_out = (long long)a.B * a.T * a.Hq;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((rows_out * 32 + 255) / 256);
+  cfg.gridDim = dim3((unsigned)((rows_out * wpr + 7) / 8));
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
@@ -651,10 +713,10 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
   const int paged_i = paged ? 1 : 0;
   if (a.d == 128)
     e = cudaLaunchKernelEx(&cfg, decode_combine_kernel<128>, (const float*)a.part_o, (const float*)a.part_lse,
-                           a.seqlens, a.o, a.o_bf16, a.lse, sp, a.B, paged_i);
+                           a.seqlens, a.o, a.o_bf16, a.lse, sp, a.B, paged_i, wpr);
   else
     e = cudaLaunchKernelEx(&cfg, decode_combine_kernel<64>, (const float*)a.part_o, (const float*)a.part_lse,
-                           a.seqlens, a.o, a.o_bf16, a.lse, sp, a.B, paged_i);
+                           a.seqlens, a.o, a.o_bf16, a.lse, sp, a.B, paged_i, wpr);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

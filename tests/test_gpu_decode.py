@@ -112,6 +112,20 @@ def test_decode_split_counts(num_splits, T):
     check_lse(lse, lse_ref)
 
 
+@pytest.mark.parametrize("num_splits,T,Hkv", [(95, 1, 2), (95, 3, 4), (6, 1, 8)])
+def test_decode_many_chunks(num_splits, T, Hkv):
+    """Up to 94 chunks of 64 keys per row (three groups of 32 LSEs to merge) and
+    chunk counts that use 1 to 8 merging warps per output row."""
+    Hq, d = 16, 128
+    lens = [6000, 64, 4097, 31]
+    case = synth.decode_inputs(len(lens), T, Hq, Hkv, d, 0, 0, seed=90 + T, device="cuda", lengths=lens)
+    host = host_copy(case)
+    o, lse = run_step(case, T, Hq, Hkv, d, 0.09, num_splits=num_splits)
+    o_ref, lse_ref = oracle_step(host, T, 0.09)
+    check_o(o, o_ref)
+    check_lse(lse, lse_ref)
+
+
 @pytest.mark.parametrize("causal", [True, False])
 def test_decode_noncausal_and_bf16_out(causal):
     T, Hq, Hkv, d = 4, 8, 2, 64
