@@ -133,3 +133,27 @@ def test_prefill_llama_workload_sampled_rows(name):
         check_lse(lse[b, h, i][None], lse_ref, f"{name} b={b} h={h} i={i}")
     del q, k, v, o, lse
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,causal", [
+    (2, 4, 2, 8200, 128, True),     # long sequences: items grouped by K/V head, ragged last block
+    (1, 4, 1, 16400, 64, True),
+    (2, 4, 2, 8192, 128, False),
+])
+def test_prefill_long_sequences_sampled_rows(B, Hq, Hkv, N, d, causal):
+    q, k, v = synth.prefill_inputs(B, Hq, Hkv, N, d, seed=12 + N, device="cuda")
+    scale = 1.0 / math.sqrt(d)
+    o, lse = run_prefill(q, k, v, scale, causal)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+    rng = np.random.default_rng(N)
+    G = Hq // Hkv
+    picks = [(int(rng.integers(B)), int(rng.integers(Hq)), int(rng.integers(N))) for _ in range(24)]
+    picks += [(0, 0, 0), (B - 1, Hq - 1, N - 1), (B - 1, 1, N - 9), (0, Hq - 1, 8191)]
+    for b, h, i in picks:
+        g = h // G
+        n_keys = i + 1 if causal else N
+        o_ref, lse_ref = oracle.attend_head(f64(q[b, i, h])[None], f64(k[b, :n_keys, g]), f64(v[b, :n_keys, g]),
+                                            scale, False)
+        check_o(o[b, i, h][None], o_ref, f"b={b} h={h} i={i}")
+        check_lse(lse[b, h, i][None], lse_ref, f"b={b} h={h} i={i}")
