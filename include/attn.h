@@ -164,7 +164,7 @@ ATTN_API size_t attn_decode_workspace_bytes(int B, int T, int Hq, int Hkv, int d
  * T may be large: a prompt chunk appended to a cached prefix (chunked prefill,
  * prefix caching; [P1] "用它" enable-prefix-caching) is this same call with T =
  * the chunk length, and T = seqlens_k[b] is a prefill from scratch.  With
- * R = (Hq / Hkv) * T query rows per KV head, R <= 32 runs on warp-level MMAs;
+ * R = (Hq / Hkv) * T query rows per KV head, R <= 16 runs on warp-level MMAs;
  * larger R on the tcgen05 tensor cores, in row tiles of whole tokens of at most
  * 128 rows, scores in TMEM.  Hq / Hkv must be <= 128.
  * Errors: ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED (d, rows per KV head),
