@@ -1,5 +1,5 @@
 // Split-KV attention of T new tokens against a KV cache on the sm_100a tensor
-// cores, for many query rows per KV head (R = (Hq/Hkv) * T above 32: grouped
+// cores, for many query rows per KV head (R = (Hq/Hkv) * T above 16: grouped
 // heads times several new tokens -- a speculative-verify step of 8 or 16
 // tokens, or a whole prompt chunk appended to an existing cache, which is
 // chunked prefill / prefill against a cached prefix).
