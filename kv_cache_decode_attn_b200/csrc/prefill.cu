@@ -108,7 +108,10 @@ enum Bar {
 };
 
 // Where K and V come from.
-enum KvSource { KV_DENSE = 0, KV_CACHE = 1, KV_PAGED = 2 };
+// KV_DENSE_GROUPED: the dense form with its items in the cached forms' order.
+enum KvSource { KV_DENSE = 0, KV_CACHE = 1, KV_PAGED = 2, KV_DENSE_GROUPED = 3 };
+template <int KV>
+constexpr bool kDenseKv = KV == KV_DENSE || KV == KV_DENSE_GROUPED;
 
 // K+V bytes of one (sequence, K/V head) of a dense prefill from which its items are
 // grouped by K/V head.  Measured on B200 (4 x 32 x 8 heads, d = 128): grouped is
@@ -126,7 +129,6 @@ struct PrefillParams {
   int B, N, Hq, Hkv, G, n_qblocks, n_ktiles, n_items;   // N: queries per sequence (Nq)
   float scale_log2;
   int causal, o_bf16;
-  int kv_major;                // dense: items grouped by (sequence, K/V head) as in the cached forms
   // cached forms only
   const int32_t* seqlens;      // [B] keys per sequence, including the N new ones
   const int32_t* page_table;   // [B, max_blocks] (paged)
@@ -152,7 +154,7 @@ struct Item {
 // Work item w.  Dense with short sequences: heaviest causal query blocks first, then
 // consecutive heads (the query heads of one K/V head are adjacent, so its K/V tiles
 // are reused from L2).  Cached forms, where sequences differ in length, and dense
-// long sequences (kv_major): sequences longest
+// long sequences (KV_DENSE_GROUPED): sequences longest
 // first (`order`, or index order when the batch is too large to rank), then K/V
 // head, then query blocks heaviest first, then the heads of that K/V head --
 // roughly longest-processing-time first, and every reader of one K/V range runs
@@ -160,7 +162,7 @@ struct Item {
 template <int KV>
 __device__ __forceinline__ Item item_of(int w, const PrefillParams& p, const int* order) {
   Item it;
-  if (KV == KV_DENSE && !p.kv_major) {
+  if constexpr (KV == KV_DENSE) {
     const int per = p.Hq * p.B;
     it.qb = p.n_qblocks - 1 - w / per;
     const int r = w - (w / per) * per;
@@ -175,7 +177,7 @@ __device__ __forceinline__ Item item_of(int w, const PrefillParams& p, const int
     it.qb = p.n_qblocks - 1 - rem2 / p.G;
     it.h = kvh * p.G + rem2 % p.G;
   }
-  if constexpr (KV == KV_DENSE) {
+  if constexpr (kDenseKv<KV>) {
     it.L = p.N;
     it.off = 0;
     it.bad = false;
@@ -208,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Q copies complete B_QFULL phase it; -1 = no more work
   volatile int* item_slot = reinterpret_cast<volatile int*>(tmem_slot + 2);
   int* order_smem = reinterpret_cast<int*>(smem + C::kOrderOff);
-  const int* order = (KV != KV_DENSE && p.B <= C::kMaxOrdered) ? order_smem : nullptr;
+  const int* order = (!kDenseKv<KV> && p.B <= C::kMaxOrdered) ? order_smem : nullptr;
   if (order) {
     // rank of each sequence by length, longest first (ties by index)
     for (int bb = threadIdx.x; bb < p.B; bb += blockDim.x) {
@@ -510,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float ls = (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
       l = l * alpha + ls;
-      if constexpr (KV != KV_DENSE) {
+      if constexpr (!kDenseKv<KV>) {
         // V rows of keys >= L: any bytes (cache) or never loaded (paged); the PV MMA
         // would multiply them by p = 0.  The group that consumes the tile last zeroes
         // them before its P arrives: tile A for j < n_kv0 (PV_A(j) is issued before
@@ -644,7 +646,7 @@ cudaError_t run_prefill(const PrefillLaunch& a, cudaStream_t stream) {
     return encode_tmap_nd(m, base, 4, dims, str, box);
   };
   if (enc(&tq, a.q, a.Hq, a.N)) return cudaErrorInvalidValue;
-  if constexpr (KV == KV_DENSE) {
+  if constexpr (kDenseKv<KV>) {
     if (enc(&tk, a.k, a.Hkv, a.N) || enc(&tv, a.v, a.Hkv, a.N)) return cudaErrorInvalidValue;
   } else if constexpr (KV == KV_CACHE) {
     if (enc(&tk, a.k, a.Hkv, a.capacity) || enc(&tv, a.v, a.Hkv, a.capacity)) return cudaErrorInvalidValue;
@@ -673,7 +675,6 @@ cudaError_t run_prefill(const PrefillLaunch& a, cudaStream_t stream) {
   p.scale_log2 = a.scale * kLog2e;
   p.causal = a.causal;
   p.o_bf16 = a.o_bf16;
-  p.kv_major = KV != KV_DENSE || 4.0 * a.N * D >= kDenseKvHeadBytes;
   p.seqlens = a.seqlens;
   p.page_table = a.page_table;
   p.max_blocks = a.max_blocks;
@@ -696,7 +697,11 @@ cudaError_t run_prefill(const PrefillLaunch& a, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_prefill(const PrefillLaunch& a, cudaStream_t stream) {
-  if (!a.seqlens) return a.d == 128 ? run_prefill<128, KV_DENSE>(a, stream) : run_prefill<64, KV_DENSE>(a, stream);
+  if (!a.seqlens) {
+    const bool grouped = 4.0 * a.N * a.d >= kDenseKvHeadBytes;
+    if (a.d == 128) return grouped ? run_prefill<128, KV_DENSE_GROUPED>(a, stream) : run_prefill<128, KV_DENSE>(a, stream);
+    return grouped ? run_prefill<64, KV_DENSE_GROUPED>(a, stream) : run_prefill<64, KV_DENSE>(a, stream);
+  }
   if (!a.page_table)
     return a.d == 128 ? run_prefill<128, KV_CACHE>(a, stream) : run_prefill<64, KV_CACHE>(a, stream);
   return a.d == 128 ? run_prefill<128, KV_PAGED>(a, stream) : run_prefill<64, KV_PAGED>(a, stream);
