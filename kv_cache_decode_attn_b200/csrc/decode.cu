@@ -465,14 +465,15 @@ __device__ __forceinline__ void accumulate(float (&acc)[kPer], float w, float4 x
 // meet in shared memory.  The sequence length is read before the wait on the split
 // kernel (that kernel does not write it); after the wait every warp issues its first
 // kBatch partial loads together with the row's LSE loads, so a row costs about two
-// dependent memory round trips.
-template <int D>
-__global__ void __launch_bounds__(256, 2) decode_combine_kernel(const float* __restrict__ part_o,
+// dependent memory round trips.  kBatch: partial loads in flight per lane -- 8 for
+// long decode (many chunks per row), 2 for launches of at most two chunks (many rows,
+// as in a prompt chunk), where a small register footprint buys five CTAs per SM.
+template <int D, int kBatch>
+__global__ void __launch_bounds__(256, kBatch >= 8 ? 2 : 5) decode_combine_kernel(const float* __restrict__ part_o,
                                                              const float* __restrict__ part_lse,
                                                              const int32_t* __restrict__ seqlens, void* o, int o_bf16,
                                                              float* lse, SplitParams p, int B, int paged, int wpr) {
   constexpr int kPer = D / 32;    // output columns per lane
-  constexpr int kBatch = 8;       // partial loads in flight per lane
   __shared__ float4 red[8][32];   // one float4 per lane of each of the 8 warps
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wi = warp & (wpr - 1);
@@ -711,12 +712,11 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const int paged_i = paged ? 1 : 0;
-  if (a.d == 128)
-    e = cudaLaunchKernelEx(&cfg, decode_combine_kernel<128>, (const float*)a.part_o, (const float*)a.part_lse,
-                           a.seqlens, a.o, a.o_bf16, a.lse, sp, a.B, paged_i, wpr);
-  else
-    e = cudaLaunchKernelEx(&cfg, decode_combine_kernel<64>, (const float*)a.part_o, (const float*)a.part_lse,
-                           a.seqlens, a.o, a.o_bf16, a.lse, sp, a.B, paged_i, wpr);
+  const bool light = sp.max_chunks <= 2;
+  auto kern = a.d == 128 ? (light ? decode_combine_kernel<128, 2> : decode_combine_kernel<128, 8>)
+                         : (light ? decode_combine_kernel<64, 2> : decode_combine_kernel<64, 8>);
+  e = cudaLaunchKernelEx(&cfg, kern, (const float*)a.part_o, (const float*)a.part_lse, a.seqlens, a.o, a.o_bf16,
+                         a.lse, sp, a.B, paged_i, wpr);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
