@@ -263,6 +263,17 @@ ATTN_API int64_t kv_cache_bytes(int n_layers, int batch, int64_t tokens, int n_k
 ATTN_API int attn_get_device_status(int clear);
 
 /*
+ * attn_selftest_wait_timeout -- check of the failure detection, not part of the
+ * pages' method.  Launches one CTA on `stream` whose thread waits on an mbarrier
+ * that nothing arrives at, through the same bounded wait every kernel of this
+ * library uses (2 s of %globaltimer, or 4e9 SM cycles, whichever ends first).
+ * The wait gives up and the kernel sets ATTN_DEV_TIMEOUT, as a kernel whose wait
+ * ran out does; attn_get_device_status then reports it and the context stays
+ * usable.  Returns ATTN_OK or ATTN_ERR_CUDA (launch failure).
+ */
+ATTN_API int attn_selftest_wait_timeout(void* stream);
+
+/*
  * attn_decode_noalloc -- attn_decode for callers that cannot allocate device
  * memory.  The pages have no counterpart: this is a packaging variant only.
  *

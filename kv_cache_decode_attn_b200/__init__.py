@@ -24,7 +24,7 @@ __all__ = [
     "attn_decode_fp8", "kv_append_fp8", "attn_prefill_cache", "BlockPool", "copy_blocks", "pool_simulate",
     "ATTN_ERR_NO_BLOCKS", "SIM_METRICS",
     "kv_cache_bytes", "ATTN_DECODE_NOALLOC_SCRATCH_BYTES",
-    "attn_get_device_status", "attn_status_string", "decode_workspace",
+    "attn_get_device_status", "attn_selftest_wait_timeout", "attn_status_string", "decode_workspace",
     "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_WORKSPACE", "ATTN_ERR_CUDA",
     "ATTN_ERR_DEVICE", "ATTN_F32", "ATTN_BF16", "ATTN_DEV_PAGE_ID", "ATTN_DEV_SEQLEN",
     "ATTN_DEV_APPEND_RANGE", "ATTN_DEV_TIMEOUT", "ATTN_DEV_SCALE",
@@ -71,6 +71,7 @@ _SIGNATURES = {
     "attn_copy_blocks": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _p]),
     "attn_pool_simulate": (_i, [_p, _i, _i64, _i, _i64, _p]),
     "attn_get_device_status": (_i, [_i]),
+    "attn_selftest_wait_timeout": (_i, [_p]),
     "attn_status_string": (ctypes.c_char_p, [_i]),
 }
 
@@ -304,6 +305,12 @@ def kv_cache_bytes(n_layers, batch, tokens, n_kv_heads, head_dim, elem_bytes) ->
 
 def attn_get_device_status(clear: bool = False) -> int:
     return int(lib.attn_get_device_status(int(bool(clear))))
+
+
+def attn_selftest_wait_timeout(stream=None) -> None:
+    """One bounded wait that nothing completes: after its limit (2 s) the device
+    status gains ``ATTN_DEV_TIMEOUT`` (read it with ``attn_get_device_status``)."""
+    _check("attn_selftest_wait_timeout", lib.attn_selftest_wait_timeout(_stream(stream)))
 
 
 # ------------------------------------------------------------------ block pool

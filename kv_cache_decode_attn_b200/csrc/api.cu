@@ -383,6 +383,13 @@ int attn_copy_blocks(void* k_pool, void* v_pool, const int32_t* src, const int32
                      "attn_copy_blocks");
 }
 
+int attn_selftest_wait_timeout(void* stream) {
+  unsigned* st = status_ptr();
+  if (!st) return ATTN_ERR_CUDA;
+  return cuda_status(launch_wait_timeout_selftest(st, static_cast<cudaStream_t>(stream)),
+                     "attn_selftest_wait_timeout");
+}
+
 int kv_append_fp8(void* k_cache, void* v_cache, const void* k_new, const void* v_new, const float* k_scale,
                   const float* v_scale, const int32_t* cache_lens, const int32_t* page_table, int max_blocks_per_seq,
                   int num_blocks, int cache_capacity, int B, int T, int Hkv, int d, void* stream) {

@@ -22,6 +22,10 @@ constexpr int kFp8MaxRows = 32;
 // Whether attn_decode runs the tensor-core split kernel for R rows per KV head.
 inline bool decode_uses_tc(int R, bool fp8) { return !fp8 && R > kDecodeMmaRows; }
 
+// One CTA whose thread waits on an mbarrier nothing arrives at (bounded like every
+// wait of the library) and then sets DEV_TIMEOUT (csrc/selftest.cu).
+cudaError_t launch_wait_timeout_selftest(unsigned* status, cudaStream_t stream);
+
 struct DecodeLaunch {
   const void* q;
   const void* k;          // contiguous cache or paged pool

@@ -21,9 +21,14 @@ enum : unsigned {
   DEV_SCALE = 16u,
 };
 
-// wall-clock limit of one bounded wait, in nanoseconds (%globaltimer)
+// wall-clock limit of one bounded wait, in nanoseconds (%globaltimer), and a
+// second, independent bound in SM clock cycles (%clock64: 2 s at 2 GHz), so that a
+// wait ends even if one of the two counters stood still
 #ifndef KVATTN_WAIT_LIMIT_NS
 #define KVATTN_WAIT_LIMIT_NS 2000000000ull
+#endif
+#ifndef KVATTN_WAIT_LIMIT_CYCLES
+#define KVATTN_WAIT_LIMIT_CYCLES 4000000000ll
 #endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -71,9 +76,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
+  const long long c0 = clock64();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0 && global_timer_ns() - t0 > KVATTN_WAIT_LIMIT_NS) return false;
+    if ((it & 255u) == 0 &&
+        (global_timer_ns() - t0 > KVATTN_WAIT_LIMIT_NS || clock64() - c0 > KVATTN_WAIT_LIMIT_CYCLES))
+      return false;
   }
 }
 
