@@ -320,7 +320,7 @@ def _sampled_rows_check(name, n_rows=12, seed=0):
     assert torch.isfinite(o).all() and torch.isfinite(lse).all()
 
 
-@pytest.mark.parametrize("name", ["decode_contig", "decode_paged", "decode_paged_t4"])
+@pytest.mark.parametrize("name", ["decode_contig", "decode_paged", "decode_paged_t4", "decode_paged_t8"])
 def test_full_size_workload_sampled_rows(name):
     _sampled_rows_check(name)
     torch.cuda.empty_cache()
