@@ -624,14 +624,16 @@ int decode_chunk_tokens(int B, int T, int G, int Hkv, int max_seqlen, int num_sp
     // balance the grid.  Measured on B200: the warp-MMA kernel (2 CTAs per SM)
     // was best at 2048 tokens for 16 x 8 sequence-heads up to 32K keys and 4096
     // for 8 x 8 up to 128K, i.e. about 14 work items per SM; the FP8 kernel for
-    // up to 8 rows (3 CTAs per SM) wants about 21; the tensor-core kernel (1 CTA
-    // per SM, a costly start) wants few long items, about 4 per SM.  Start long
-    // and halve until the grid holds that many items (counted as if every
-    // sequence had max_seqlen; row tiles of many new tokens count separately).
+    // up to 8 rows (3 CTAs per SM) wants about 21; the tensor-core kernel
+    // (2 CTAs per SM) about 9 for row tiles of up to 64 rows and about 4 for full
+    // 128-row tiles, whose softmax makes each tile dearer.  Start long and halve
+    // until the grid holds that many items (counted as if every sequence had
+    // max_seqlen; row tiles of many new tokens count separately).
     const int R = G * T;
     const bool tc = decode_uses_tc(R, fp8);
     const long long units = (long long)B * Hkv * decode_row_tiles(T, G);
-    const long long target = tc ? 640 : (fp8 && R <= 8 ? 3072 : 2048);
+    const bool full_tiles = decode_tc_tile_tokens(T, G) * G > 64;
+    const long long target = tc ? (full_tiles ? 640 : 1280) : (fp8 && R <= 8 ? 3072 : 2048);
     chunk = tc ? 16384 : 4096;
     while (chunk > 256 && units * ((max_seqlen + chunk - 1) / chunk) < target) chunk >>= 1;
   }

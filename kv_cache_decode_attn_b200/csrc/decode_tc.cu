@@ -13,8 +13,8 @@
 //   warps 0..3  softmax: thread i owns row i (TMEM lane i); warps whose rows are
 //               all >= R stay idle;
 //   warps 4, 6  TMA producers: warp 4 loads Q once and the K tiles, warp 6 the V
-//               tiles, each into its own 3-stage ring with the evict-first L2
-//               policy (128-token tiles; contiguous: one 128-row box per 64
+//               tiles, each into its own 2-stage ring with the evict-first L2
+//               policy (64-token tiles; contiguous: one 64-row box per 64
 //               columns of d; paged: one 16-row box per physical block, its
 //               page-table entry checked first).  K is released by S_j, V only by
 //               PV_j, so separate producers let the K ring run ahead;
@@ -24,6 +24,9 @@
 //               tensor core computes the next scores while the softmax runs.
 // Online softmax with the lazy rescale of the prefill kernel: a row's reference
 // maximum is raised only when a tile's maximum exceeds it by more than 8.
+// 64-token tiles keep a CTA at 99.6 KB of shared memory and 256 TMEM columns, so
+// two CTAs share an SM: one streams while the other starts up or writes its
+// partials, and the grid's last wave is split over twice as many slots.
 //
 // Method: "[BEE-30062] FlashAttention 與高效注意力核心", "背景" and
 // "為長上下文推論啟用 FlashDecoding" (split along the KV length, stable merge of
@@ -40,24 +43,28 @@ namespace kvattn {
 namespace {
 
 constexpr int kRows = 128;   // MMA M (query rows per KV head, padded)
-constexpr int kTok = 128;    // keys per K/V tile
+constexpr int kTok = kDecodeTcTile;   // keys per K/V tile (the host's tensor-map box)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-constexpr int kStages = 3;    // K/V ring stages (S is double-buffered in TMEM)
+constexpr int kStages = 2;    // K/V ring stages (S is double-buffered in TMEM)
+constexpr int kCtasPerSm = 2;   // shared memory and TMEM of one CTA
 
 template <int D>
 struct TcCfg {
   static constexpr int kHalves = D / 64;
-  static constexpr int kHalfBytes = kTok * 128;              // 128 rows x 128 B
-  static constexpr int kTileBytes = kTok * D * 2;            // one K or V tile (= the Q tile)
+  static constexpr int kQHalfBytes = kRows * 128;            // Q: 128 rows x 128 B per 64 columns of d
+  static constexpr int kHalfBytes = kTok * 128;              // K or V tile: kTok rows x 128 B
+  static constexpr int kQBytes = kRows * D * 2;
+  static constexpr int kTileBytes = kTok * D * 2;            // one K or V tile
   static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + kTileBytes;           // K stages
+  static constexpr int kKOff = kQOff + kQBytes;              // K stages
   static constexpr int kVOff = kKOff + kStages * kTileBytes; // V stages
   static constexpr int kBarOff = kVOff + kStages * kTileBytes;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;
-  static constexpr int kTmemCols = 512;                      // S0 | S1 | O (+ unused)
-  static constexpr int kOCol = 256;
+  static constexpr int kSCols = kTok;                        // one S buffer (fp32 scores of a tile)
+  static constexpr int kOCol = 2 * kSCols;                   // S0 | S1 | O
+  static constexpr int kTmemCols = kOCol + D <= 256 ? 256 : 512;
 };
 
 // K and V stages are released separately: K_j as soon as S_j is done, V_j once PV_j is done.
@@ -105,7 +112,7 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
 }
 
 template <int D, bool PAGED>
-__global__ void __launch_bounds__(224, 1)
+__global__ void __launch_bounds__(224, kCtasPerSm)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const TcParams p) {
   using C = TcCfg<D>;
@@ -165,7 +172,7 @@ __global__ void __launch_bounds__(224, 1)
     const int per_half = (kRows - box_rows) * 8;   // 16-byte chunks of rows box_rows..127 in one half of d
     for (int i = threadIdx.x; i < per_half * C::kHalves; i += blockDim.x) {
       const int half = i / per_half, rem = i - half * per_half;
-      *reinterpret_cast<uint4*>(smem + C::kQOff + half * C::kHalfBytes + box_rows * 128 + rem * 16) =
+      *reinterpret_cast<uint4*>(smem + C::kQOff + half * C::kQHalfBytes + box_rows * 128 + rem * 16) =
           make_uint4(0, 0, 0, 0);
     }
   }
@@ -192,7 +199,7 @@ __global__ void __launch_bounds__(224, 1)
         mbar_arrive_expect_tx(&bars[T_Q], p.TT * p.G * D * 2);
 #pragma unroll
         for (int hh = 0; hh < C::kHalves; ++hh)
-          tma_load_4d(smem + C::kQOff + hh * C::kHalfBytes, &tmQ, &bars[T_Q], hh * 64, g * p.G, t0, b, pol);
+          tma_load_4d(smem + C::kQOff + hh * C::kQHalfBytes, &tmQ, &bars[T_Q], hh * 64, g * p.G, t0, b, pol);
       }
       uint8_t* ring = smem + (is_k ? C::kKOff : C::kVOff);
       const int full0 = is_k ? T_KFULL : T_VFULL, empty0 = is_k ? T_KEMPTY : T_VEMPTY;
@@ -216,7 +223,7 @@ __global__ void __launch_bounds__(224, 1)
           }
         return nb;
       };
-      int ids[kBlocks] = {0, 0, 0, 0, 0, 0, 0, 0};
+      int ids[kBlocks] = {};
       int nb = PAGED ? read_ids(0, ids) : 0;
       for (int i = 0; i < n_tiles; ++i) {
         const int ks = i % kStages;
@@ -259,8 +266,10 @@ __global__ void __launch_bounds__(224, 1)
         const uint32_t k_s = smem_u32(smem + C::kKOff + ks * C::kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
-          tc_mma_ss(tmem + sb * 128, smem_desc(q_s + off, 16, 1024), smem_desc(k_s + off, 16, 1024), idS, kk > 0);
+          const uint32_t q_off = (kk >> 2) * C::kQHalfBytes + (kk & 3) * 32;
+          const uint32_t k_off = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
+          tc_mma_ss(tmem + sb * C::kSCols, smem_desc(q_s + q_off, 16, 1024), smem_desc(k_s + k_off, 16, 1024), idS,
+                    kk > 0);
         }
         tc_commit(&bars[T_SFULL + sb]);
         tc_commit(&bars[T_KEMPTY + ks]);     // K_i is read only by S_i
@@ -286,7 +295,7 @@ __global__ void __launch_bounds__(224, 1)
         const uint32_t v_s = smem_u32(smem + C::kVOff + ks * C::kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < kTok / 16; ++kk)
-          tc_mma_ts(tmem + C::kOCol, tmem + sb * 128 + kk * 8, smem_desc(v_s + kk * 16 * 128, C::kHalfBytes, 1024),
+          tc_mma_ts(tmem + C::kOCol, tmem + sb * C::kSCols + kk * 8, smem_desc(v_s + kk * 16 * 128, C::kHalfBytes, 1024),
                     idO, (i > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&bars[T_ODONE]);
         tc_commit(&bars[T_VEMPTY + ks]);
@@ -307,7 +316,7 @@ __global__ void __launch_bounds__(224, 1)
       const int st = i & 1;
       if (!tc_wait(&bars[T_SFULL + st], (i >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t s_addr = lane_base + st * 128;
+      const uint32_t s_addr = lane_base + st * C::kSCols;
       float s[kTok];
 #pragma unroll
       for (int cc = 0; cc < kTok; cc += 32) {

@@ -10,7 +10,7 @@ namespace kvattn {
 
 constexpr int kPageTokens = 16;   // tokens per physical KV block
 constexpr int kDecodeTile = 64;   // tokens per pipeline stage of the warp-MMA decode kernel
-constexpr int kDecodeTcTile = 128;  // tokens per K/V tile of the tensor-core decode kernel
+constexpr int kDecodeTcTile = 64;  // tokens per K/V tile of the tensor-core decode kernel
 // Above this many query rows per KV head the tensor-core kernel runs (bf16
 // caches).  Measured on B200 (paged Llama decode, 8 KV heads x 8 sequences):
 // 32 rows ran at 5.7 TB/s there against 4.5 TB/s on the warp-MMA kernel, whose
