@@ -257,52 +257,57 @@ __global__ void __launch_bounds__(224, kCtasPerSm)
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(kRows, kTok, 0, 0);
-      constexpr uint32_t idO = idesc_bf16(kRows, D, 0, 1);
-      const uint32_t q_s = smem_u32(smem + C::kQOff);
-      auto issue_s = [&](int i) {
-        const int sb = i & 1, ks = i % kStages;   // S buffer, K/V ring stage
-        const uint32_t k_s = smem_u32(smem + C::kKOff + ks * C::kTileBytes);
+    // The whole warp runs the loop (warp-uniform operands, descriptors as precomputed
+    // low words plus compile-time offsets); one elected lane issues and commits.
+    const uint32_t leader = elect_one();
+    constexpr uint32_t idS = idesc_bf16(kRows, kTok, 0, 0);
+    constexpr uint32_t idO = idesc_bf16(kRows, D, 0, 1);
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t q_lo = desc_lo(sbase + C::kQOff, 16);
+    auto issue_s = [&](int i) {
+      const int sb = i & 1, ks = i % kStages;   // S buffer, K/V ring stage
+      const uint32_t k_lo = desc_lo(sbase + C::kKOff + ks * C::kTileBytes, 16);
+      const uint32_t d = tmem + sb * C::kSCols;
+      tc_mma_ss_lo<0>(leader, d, q_lo, k_lo, idS);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t q_off = (kk >> 2) * C::kQHalfBytes + (kk & 3) * 32;
-          const uint32_t k_off = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
-          tc_mma_ss(tmem + sb * C::kSCols, smem_desc(q_s + q_off, 16, 1024), smem_desc(k_s + k_off, 16, 1024), idS,
-                    kk > 0);
-        }
-        tc_commit(&bars[T_SFULL + sb]);
-        tc_commit(&bars[T_KEMPTY + ks]);     // K_i is read only by S_i
-      };
-      bool ok = tc_wait(&bars[T_Q], 0, abort_flag, p.status) &&
-                tc_wait(&bars[T_KFULL], 0, abort_flag, p.status);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0);
+      for (int kk = 1; kk < D / 16; ++kk) {
+        const uint32_t q_off = ((kk >> 2) * C::kQHalfBytes + (kk & 3) * 32) >> 4;
+        const uint32_t k_off = ((kk >> 2) * C::kHalfBytes + (kk & 3) * 32) >> 4;
+        tc_mma_ss_lo<1>(leader, d, q_lo + q_off, k_lo + k_off, idS);
       }
-      for (int i = 0; ok && i < n_tiles; ++i) {
-        const int sb = i & 1, ks = i % kStages;
-        if (i + 1 < n_tiles) {
-          ok = tc_wait(&bars[T_KFULL + (i + 1) % kStages], ((i + 1) / kStages) & 1, abort_flag, p.status);
-          if (!ok) break;
-          tc_fence_after();
-          issue_s(i + 1);   // its S buffer last held P_{i-1}, whose PV was issued before
-        }
-        ok = tc_wait(&bars[T_PFULL + sb], (i >> 1) & 1, abort_flag, p.status) &&
-             tc_wait(&bars[T_VFULL + ks], (i / kStages) & 1, abort_flag, p.status);
+      tc_commit_if(leader, &bars[T_SFULL + sb]);
+      tc_commit_if(leader, &bars[T_KEMPTY + ks]);     // K_i is read only by S_i
+    };
+    bool ok = tc_wait(&bars[T_Q], 0, abort_flag, p.status) &&
+              tc_wait(&bars[T_KFULL], 0, abort_flag, p.status);
+    if (ok) {
+      tc_fence_after();
+      issue_s(0);
+    }
+    for (int i = 0; ok && i < n_tiles; ++i) {
+      const int sb = i & 1, ks = i % kStages;
+      if (i + 1 < n_tiles) {
+        ok = tc_wait(&bars[T_KFULL + (i + 1) % kStages], ((i + 1) / kStages) & 1, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t v_s = smem_u32(smem + C::kVOff + ks * C::kTileBytes);
-#pragma unroll
-        for (int kk = 0; kk < kTok / 16; ++kk)
-          tc_mma_ts(tmem + C::kOCol, tmem + sb * C::kSCols + kk * 8, smem_desc(v_s + kk * 16 * 128, C::kHalfBytes, 1024),
-                    idO, (i > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&bars[T_ODONE]);
-        tc_commit(&bars[T_VEMPTY + ks]);
+        issue_s(i + 1);   // its S buffer last held P_{i-1}, whose PV was issued before
       }
-      // also on a failed wait, so that the epilogue does not wait in vain (abort_flag marks the result)
-      tc_commit(&bars[T_OFINAL]);
+      ok = tc_wait(&bars[T_PFULL + sb], (i >> 1) & 1, abort_flag, p.status) &&
+           tc_wait(&bars[T_VFULL + ks], (i / kStages) & 1, abort_flag, p.status);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t v_lo = desc_lo(sbase + C::kVOff + ks * C::kTileBytes, C::kHalfBytes);
+      const uint32_t d = tmem + C::kOCol, pa = tmem + sb * C::kSCols;
+      if (i == 0) tc_mma_ts_lo<0>(leader, d, pa, v_lo, idO);
+      else tc_mma_ts_lo<1>(leader, d, pa, v_lo, idO);
+#pragma unroll
+      for (int kk = 1; kk < kTok / 16; ++kk)
+        tc_mma_ts_lo<1>(leader, d, pa + kk * 8, v_lo + ((kk * 16 * 128) >> 4), idO);
+      tc_commit_if(leader, &bars[T_ODONE]);
+      tc_commit_if(leader, &bars[T_VEMPTY + ks]);
     }
+    // also on a failed wait, so that the epilogue does not wait in vain (abort_flag marks the result)
+    tc_commit_if(leader, &bars[T_OFINAL]);
   } else if (warp < active_warps) {
     // ------------------------------------------------------------- softmax warps
     const int row = warp * 32 + lane;
@@ -427,8 +432,10 @@ __global__ void __launch_bounds__(224, kCtasPerSm)
 
   tc_fence_before();
   __syncthreads();
-  if (*abort_flag && warp == 5 && lane == 0) {
-    tc_commit(&bars[T_DRAIN]);
+  if (*abort_flag && warp == 5) {
+    // the lane that issued the MMAs commits, so the drain covers them
+    const uint32_t leader = elect_one();
+    tc_commit_if(leader, &bars[T_DRAIN]);
     mbar_wait(&bars[T_DRAIN], 0);
   }
   __syncthreads();

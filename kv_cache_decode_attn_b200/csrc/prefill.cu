@@ -5,16 +5,23 @@
 // a ticket from a global counter, so a CTA that finishes early takes more
 // work instead of waiting on a fixed share).  A work item is two 128-row query tiles (A: rows 256*qb .. +127,
 // B: the next 128) of one (batch, query head); both tiles share every K/V tile
-// loaded for the item.  Warp roles:
+// loaded for the item.  Warp roles (12 warps, three warpgroups):
 //   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread i of a
 //              group owns query row i, which is TMEM lane i of its S and O;
 //   warp 8     TMA producer: Q_A and Q_B per item (the next item's Q is
 //              prefetched into L2 early), K_j and V_j through a 2-stage ring
-//              that runs on across items;
-//   warp 9     MMA issuer (one thread).
+//              that runs on across items; K and V of a stage are released
+//              separately (K after the second S MMA, V after the second PV);
+//   warp 9     MMA issuer: the whole warp runs the loop, one elected lane
+//              issues (operands stay warp-uniform, so each MMA costs the
+//              issuing warp only a few instructions on a sub-partition it
+//              shares with two busy softmax warps);
+//   warps 10-11 complete the producer warpgroup for the register split.
 // TMEM (512 columns): S_A | S_B | O_A | O_B.  Each softmax group reads its S row,
 // turns it into bf16 probabilities P and writes P back over the first half of
-// the same S columns; the PV MMA reads P straight from TMEM as its A operand.
+// the same S columns, in two halves of 64 keys: the PV MMA of the first half
+// (reading P straight from TMEM as its A operand) is issued while the group
+// computes the second.
 // The MMA issue order  PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), PV_A(j+1), ...
 // gives each softmax group the time of two MMAs to produce its next P.  Because
 // MMAs complete in issue order, "S_X(j) complete" also means "PV_X(j-1)
@@ -68,7 +75,13 @@ namespace {
 
 constexpr int kBM = 128;          // query rows per tile (two tiles per CTA)
 constexpr int kBN = 128;          // keys per K/V tile
-constexpr int kThreads = 320;     // 8 softmax warps + TMA warp + MMA warp
+constexpr int kThreads = 384;     // 8 softmax warps + TMA warp + MMA warp + 2 idle warps (a full warpgroup)
+// Register split (setmaxnreg): 384 threads launch with 168 registers each; the producer
+// warpgroup (TMA, MMA, two idle warps) gives back down to kRegsIo so each softmax thread
+// can hold its 128 scores and the exponential temporaries without spilling.
+constexpr int kRegsIo = 72;
+constexpr int kRegsSoftmax = 216;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsIo <= 168 * kThreads, "register split exceeds the launch");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 of the largest allowed p
@@ -98,13 +111,15 @@ enum Bar {
   B_QEMPTY = 1,   // all MMAs of an item done: its Q tiles may be replaced
   B_KFULL = 2,    // +stage
   B_VFULL = 4,    // +stage
-  B_KVEMPTY = 6,  // +stage
-  B_SFULL = 8,    // +tile
-  B_PFULL = 10,   // +tile
-  B_ODONE = 12,   // +tile: last PV of an item done
-  B_OFREE = 14,   // +tile: the softmax group has read O out
-  B_DRAIN = 16,   // only used when a bounded wait gave up
-  B_COUNT = 17
+  B_KEMPTY = 6,   // +stage: both S MMAs reading this K stage are done
+  B_VEMPTY = 8,   // +stage: both PV MMAs reading this V stage are done
+  B_SFULL = 10,   // +tile
+  B_PHALF = 12,   // +tile: P of the tile's first 64 keys is in TMEM (and O is rescaled)
+  B_PFULL = 14,   // +tile: P of all 128 keys is in TMEM
+  B_ODONE = 16,   // +tile: last PV of an item done
+  B_OFREE = 18,   // +tile: the softmax group has read O out
+  B_DRAIN = 20,   // only used when a bounded wait gave up
+  B_COUNT = 21
 };
 
 // Where K and V come from.
@@ -196,6 +211,60 @@ __device__ __forceinline__ Item item_of(int w, const PrefillParams& p, const int
   return it;
 }
 
+// 2^x for two values on the FMA pipe (no SFU): x = n + f with n = round(x) (the
+// "magic number" 1.5 * 2^23 rounds to the nearest integer), 2^f on [-1/2, 1/2] by a
+// cubic fitted for minimax relative error (7.5e-5, far below the 2^-9 of the bf16 P it
+// feeds), and 2^n added to the exponent field.  x is clamped to [-126, +inf): scores
+// reach here relative to the running maximum (x <= 8), and below -126 the true value
+// (< 1.2e-38) is replaced by a denormal of about that size.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  constexpr float kMagic = 12582912.f;
+  constexpr float kC0 = 0.99992807f, kC1 = 0.69326097f, kC2 = 0.24261113f, kC3 = 0.055171669f;
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = __fadd2_rn(x, make_float2(kMagic, kMagic));            // low bits hold n
+  const float2 n = __fadd2_rn(t, make_float2(-kMagic, -kMagic));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);             // x - n, exact
+  float2 q = __ffma2_rn(f, make_float2(kC3, kC3), make_float2(kC2, kC2));
+  q = __ffma2_rn(q, f, make_float2(kC1, kC1));
+  q = __ffma2_rn(q, f, make_float2(kC0, kC0));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// Which pairs of each 16-key group take the FMA-pipe exponential (bit i: keys 2i, 2i+1).
+// The SFU issues 16 exponentials per clock per SM, so a 128 x 128 score tile alone costs
+// as much SFU time as its two MMAs at d = 128, and twice as much at d = 64.  Measured on
+// B200: at d = 128 the extra FMA-pipe instructions cost more than the SFU time they
+// save (the softmax warps share their sub-partitions' issue slots with the MMA warp),
+// so every exponential stays on the SFU; at d = 64, three pairs in eight (37.5 %) on the
+// FMA pipe gained 3-4 % on the GPT-2-sized prefill.
+template <int D>
+constexpr unsigned exp_fma_pairs() { return D == 64 ? 0x92u : 0u; }
+
+// Exponentials of keys 64*HALF .. 64*HALF+63 of one row: p = 2^(s*sc - m) (nm = -m), the
+// pair sums added to sum2, and bf16 P stored to TMEM at taddr (two keys per column).
+// FMA: use the FMA-pipe exponential on the pairs kExpFmaPairs selects (rows without
+// masked keys only; no pair when it is 0).
+template <int HALF, bool FMA, unsigned kExpFmaPairs>
+__device__ __forceinline__ void exp_store_half(const float (&s)[kBN], float2 sc, float2 nm, float2 (&sum2)[4],
+                                               uint32_t taddr) {
+#pragma unroll
+  for (int c = HALF * (kBN / 2); c < (HALF + 1) * (kBN / 2); c += 16) {
+    uint32_t pk[8];
+#pragma unroll
+    for (int e = 0; e < 16; e += 2) {
+      const float2 x = __ffma2_rn(make_float2(s[c + e], s[c + e + 1]), sc, nm);
+      float2 pr;
+      if (FMA && ((kExpFmaPairs >> (e / 2)) & 1u)) pr = exp2_fma2(x);
+      else pr = make_float2(ex2(x.x), ex2(x.y));
+      sum2[(e >> 1) & 3] = __fadd2_rn(sum2[(e >> 1) & 3], pr);
+      pk[e / 2] = pack_bf16x2(pr.x, pr.y);
+    }
+    tmem_st8(taddr + c / 2, pk);
+  }
+}
+
 template <int D, int KV>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -232,8 +301,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[B_KFULL + s], 1);
       mbar_init(&bars[B_VFULL + s], 1);
-      mbar_init(&bars[B_KVEMPTY + s], 1);
+      mbar_init(&bars[B_KEMPTY + s], 1);
+      mbar_init(&bars[B_VEMPTY + s], 1);
       mbar_init(&bars[B_SFULL + s], 1);
+      mbar_init(&bars[B_PHALF + s], 4);
       mbar_init(&bars[B_PFULL + s], 4);
       mbar_init(&bars[B_ODONE + s], 1);
       mbar_init(&bars[B_OFREE + s], 4);
@@ -250,7 +321,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
+  if (warp >= 8) {
+  reg_dealloc<kRegsIo>();
   if (warp == 8) {
     // ------------------------------------------------------------- TMA producer
     if (lane == 0) {
@@ -260,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t keep = policy_evict_last();    // K/V tiles are re-read by other query blocks and heads
       const uint64_t once = policy_evict_first();
       int g = 0, it = 0, q_loaded = 0;              // K/V tiles loaded, items started, Q loads issued
-      int last_g[2] = {-1, -1};
+      int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};   // last K / V tile whose copy was issued per stage
       bool ok = true, clean_end = false;
       for (int w = blockIdx.x;; ++it) {
         // Q of the previous item no longer read (this also means its copy landed)
@@ -305,17 +377,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (KV == KV_PAGED) read_ids(0);
         for (int t = 0; t < itm.n_load; ++t, ++g) {
           const int st = g & 1;
-          if (g >= 2 && !wait_or_abort(&bars[B_KVEMPTY + st], ((g >> 1) - 1) & 1, abort_flag, p.status)) {
+          // K of this stage is released after the second S MMA reading it, V after the
+          // second PV MMA, so the next K tile lands while the current PVs still run
+          if (g >= 2 && !wait_or_abort(&bars[B_KEMPTY + st], ((g >> 1) - 1) & 1, abort_flag, p.status)) {
             ok = false;
             break;
           }
-          last_g[st] = g;
+          last_k[st] = g;
           if constexpr (KV != KV_PAGED) {
             mbar_arrive_expect_tx(&bars[B_KFULL + st], C::kTileBytes);
 #pragma unroll
             for (int hh = 0; hh < C::kHalves; ++hh)
               tma_load_4d(smem + C::kKOff + st * C::kTileBytes + hh * C::kHalfBytes, &tmK, &bars[B_KFULL + st],
                           hh * 64, kvh, t * kBN, itm.b, keep);
+            if (g >= 2 && !wait_or_abort(&bars[B_VEMPTY + st], ((g >> 1) - 1) & 1, abort_flag, p.status)) {
+              ok = false;
+              break;
+            }
+            last_v[st] = g;
             mbar_arrive_expect_tx(&bars[B_VFULL + st], C::kTileBytes);
 #pragma unroll
             for (int hh = 0; hh < C::kHalves; ++hh)
@@ -340,6 +419,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_load_3d(smem + C::kKOff + st * C::kTileBytes + hh * C::kHalfBytes + jb * kPageTokens * 128, &tmK,
                             &bars[B_KFULL + st], hh * 64, kvh, ids[jb] * kPageTokens, keep);
             }
+            if (g >= 2 && !wait_or_abort(&bars[B_VEMPTY + st], ((g >> 1) - 1) & 1, abort_flag, p.status)) {
+              ok = false;
+              break;
+            }
+            last_v[st] = g;
             mbar_arrive_expect_tx(&bars[B_VFULL + st], bytes);
 #pragma unroll
             for (int jb = 0; jb < kBlocks; ++jb) {
@@ -359,85 +443,114 @@ __global__ void __launch_bounds__(kThreads, 1)
       // end, the wait on B_QEMPTY above already covered the last Q copy)
       if (!clean_end && q_loaded > 0) mbar_wait(&bars[B_QFULL], (q_loaded - 1) & 1);
       for (int st = 0; st < 2; ++st) {
-        if (last_g[st] < 0) continue;
-        mbar_wait(&bars[B_KFULL + st], (last_g[st] >> 1) & 1);
-        mbar_wait(&bars[B_VFULL + st], (last_g[st] >> 1) & 1);
+        if (last_k[st] >= 0) mbar_wait(&bars[B_KFULL + st], (last_k[st] >> 1) & 1);
+        if (last_v[st] >= 0) mbar_wait(&bars[B_VFULL + st], (last_v[st] >> 1) & 1);
       }
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(kBM, kBN, 0, 0);     // Q (K-major) x K^T (K-major)
-      constexpr uint32_t idO = idesc_bf16(kBM, D, 0, 1);       // P (TMEM) x V (N-major)
-      auto issue_s = [&](int t, int st) {     // S_t = Q_t K^T, K in ring stage st
-        const uint32_t q_s = smem_u32(smem + C::kQOff + t * C::kTileBytes);
-        const uint32_t k_s = smem_u32(smem + C::kKOff + st * C::kTileBytes);
+    // The whole warp runs this loop and its waits, so that every operand (descriptors,
+    // stages, item sizes) is warp-uniform; one elected lane issues the MMAs and commits.
+    // Issued from a single divergent lane, each MMA cost about 110 clock cycles of
+    // issue on a sub-partition shared with two softmax warps -- more than its 64 cycles
+    // of tensor-core time.
+    const uint32_t leader = elect_one();
+    constexpr uint32_t idS = idesc_bf16(kBM, kBN, 0, 0);     // Q (K-major) x K^T (K-major)
+    constexpr uint32_t idO = idesc_bf16(kBM, D, 0, 1);       // P (TMEM) x V (N-major)
+    // shared-memory descriptors (128-byte swizzle, 1024-byte row-group stride): only the
+    // low word varies -- the start address in 16-byte units -- so every operand is a
+    // precomputed base (Q tile, K or V ring stage) plus a compile-time K-step offset
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t q_lo0 = desc_lo(sbase + C::kQOff, 16), q_lo1 = desc_lo(sbase + C::kQOff + C::kTileBytes, 16);
+    const uint32_t k_lo0 = desc_lo(sbase + C::kKOff, 16), k_lo1 = desc_lo(sbase + C::kKOff + C::kTileBytes, 16);
+    const uint32_t v_lo0 = desc_lo(sbase + C::kVOff, C::kHalfBytes);
+    const uint32_t v_lo1 = desc_lo(sbase + C::kVOff + C::kTileBytes, C::kHalfBytes);
+    auto issue_s = [&](int t, int st) {     // S_t = Q_t K^T, K in ring stage st
+      const uint32_t qa = t ? q_lo1 : q_lo0, kb = st ? k_lo1 : k_lo0;
+      const uint32_t d = tmem + C::s_col(t);
+      tc_mma_ss_lo<0>(leader, d, qa, kb, idS);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
-          tc_mma_ss(tmem + C::s_col(t), smem_desc(q_s + off, 16, 1024), smem_desc(k_s + off, 16, 1024), idS, kk > 0);
-        }
-        tc_commit(&bars[B_SFULL + t]);
-      };
-      auto issue_pv = [&](int t, int st, bool first) {   // O_t (+)= P_t V, P_t in the first 64 columns of S_t
-        const uint32_t v_s = smem_u32(smem + C::kVOff + st * C::kTileBytes);
+      for (int kk = 1; kk < D / 16; ++kk) {
+        const uint32_t off = ((kk >> 2) * C::kHalfBytes + (kk & 3) * 32) >> 4;
+        tc_mma_ss_lo<1>(leader, d, qa + off, kb + off, idS);
+      }
+      tc_commit_if(leader, &bars[B_SFULL + t]);
+    };
+    // O_t (+)= P_t V over keys 64*half .. 64*half+63; P_t sits in the first 64 columns of S_t
+    auto issue_pv = [&](int t, int st, bool first, int half) {
+      const uint32_t vb = st ? v_lo1 : v_lo0;
+      const uint32_t d = tmem + C::o_col(t), pa = tmem + C::s_col(t);
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          tc_mma_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8, smem_desc(v_s + kk * 16 * 128, C::kHalfBytes, 1024),
-                    idO, (!first || kk > 0) ? 1u : 0u);
-      };
-      int g = 0, it = 0;                     // K/V tiles consumed, items done
-      int pcnt[2] = {0, 0};                  // P_FULL phases consumed per tile
-      bool ok = true;
-      for (;; ++it) {
-        if (!wait_or_abort(&bars[B_QFULL], it & 1, abort_flag, p.status)) break;
-        const int w = item_slot[it & 1];
-        if (w < 0) break;                    // no more work
-        const Item itm = item_of<KV>(w, p, order);
-        const int g0 = g;
-        ok = wait_or_abort(&bars[B_KFULL + (g0 & 1)], (g0 >> 1) & 1, abort_flag, p.status);
+      for (int k4 = 0; k4 < kBN / 32; ++k4) {
+        const int kk = half * (kBN / 32) + k4;
+        if (kk == 0 && first) tc_mma_ts_lo<0>(leader, d, pa, vb, idO);
+        else tc_mma_ts_lo<1>(leader, d, pa + kk * 8, vb + ((kk * 16 * 128) >> 4), idO);
+      }
+    };
+    int pcnt[2] = {0, 0};                  // P phases consumed per tile
+    // both halves of PV_t(j): the first as soon as the softmax group has published P of
+    // the first 64 keys (the second half's exponentials overlap it)
+    auto pv_tile = [&](int t, int st, int j, int it) -> bool {
+      const uint32_t par = (pcnt[t]++) & 1;
+      if (!wait_or_abort(&bars[B_PHALF + t], par, abort_flag, p.status)) return false;
+      if (j == 0 && it > 0 && !wait_or_abort(&bars[B_OFREE + t], (it - 1) & 1, abort_flag, p.status)) return false;
+      tc_fence_after();
+      issue_pv(t, st, j == 0, 0);
+      if (!wait_or_abort(&bars[B_PFULL + t], par, abort_flag, p.status)) return false;
+      tc_fence_after();
+      issue_pv(t, st, j == 0, 1);
+      return true;
+    };
+    int g = 0, it = 0;                     // K/V tiles consumed, items done
+    bool ok = true;
+    for (;; ++it) {
+      if (!wait_or_abort(&bars[B_QFULL], it & 1, abort_flag, p.status)) break;
+      const int w = __shfl_sync(0xffffffffu, item_slot[it & 1], 0);
+      if (w < 0) break;                    // no more work
+      const Item itm = item_of<KV>(w, p, order);
+      const int n_load = __shfl_sync(0xffffffffu, itm.n_load, 0);
+      const int n_kv0 = __shfl_sync(0xffffffffu, itm.n_kv0, 0);
+      const int g0 = g;
+      ok = wait_or_abort(&bars[B_KFULL + (g0 & 1)], (g0 >> 1) & 1, abort_flag, p.status);
+      if (!ok) break;
+      tc_fence_after();
+      issue_s(0, g0 & 1);
+      issue_s(1, g0 & 1);
+      tc_commit_if(leader, &bars[B_KEMPTY + (g0 & 1)]);
+      for (int j = 0; j < n_load; ++j) {
+        const int gj = g0 + j, st = gj & 1;
+        const bool next_k = j + 1 < n_load;
+        ok = wait_or_abort(&bars[B_VFULL + st], (gj >> 1) & 1, abort_flag, p.status);
         if (!ok) break;
-        tc_fence_after();
-        issue_s(0, g0 & 1);
-        issue_s(1, g0 & 1);
-        for (int j = 0; j < itm.n_load; ++j) {
-          const int gj = g0 + j, st = gj & 1;
-          const bool next_k = j + 1 < itm.n_load;
-          ok = wait_or_abort(&bars[B_VFULL + st], (gj >> 1) & 1, abort_flag, p.status);
+        if (j < n_kv0) {
+          ok = pv_tile(0, st, j, it);
           if (!ok) break;
-          if (j < itm.n_kv0) {
-            ok = wait_or_abort(&bars[B_PFULL + 0], (pcnt[0]++) & 1, abort_flag, p.status) &&
-                 (j > 0 || it == 0 || wait_or_abort(&bars[B_OFREE + 0], (it - 1) & 1, abort_flag, p.status));
-            if (!ok) break;
-            tc_fence_after();
-            issue_pv(0, st, j == 0);
-            if (j == itm.n_kv0 - 1) tc_commit(&bars[B_ODONE + 0]);
-          }
-          if (next_k) {
-            ok = wait_or_abort(&bars[B_KFULL + ((gj + 1) & 1)], ((gj + 1) >> 1) & 1, abort_flag, p.status);
-            if (!ok) break;
-            tc_fence_after();
-            if (j + 1 < itm.n_kv0) issue_s(0, (gj + 1) & 1);
-          }
-          ok = wait_or_abort(&bars[B_PFULL + 1], (pcnt[1]++) & 1, abort_flag, p.status) &&
-               (j > 0 || it == 0 || wait_or_abort(&bars[B_OFREE + 1], (it - 1) & 1, abort_flag, p.status));
+          if (j == n_kv0 - 1) tc_commit_if(leader, &bars[B_ODONE + 0]);
+        }
+        if (next_k) {
+          ok = wait_or_abort(&bars[B_KFULL + ((gj + 1) & 1)], ((gj + 1) >> 1) & 1, abort_flag, p.status);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(1, st, j == 0);
-          tc_commit(&bars[B_KVEMPTY + st]);       // K and V of this stage are no longer needed
-          if (j == itm.n_load - 1) tc_commit(&bars[B_ODONE + 1]);
-          if (next_k) {
-            issue_s(1, (gj + 1) & 1);
-            // that was the item's last MMA reading Q: the next item's Q may land once it is done
-            if (j + 2 == itm.n_load) tc_commit(&bars[B_QEMPTY]);
-          }
+          if (j + 1 < n_kv0) issue_s(0, (gj + 1) & 1);
         }
+        ok = pv_tile(1, st, j, it);
         if (!ok) break;
-        if (itm.n_load == 1) tc_commit(&bars[B_QEMPTY]);
-        g = g0 + itm.n_load;
+        tc_commit_if(leader, &bars[B_VEMPTY + st]);        // V of this stage is no longer needed
+        if (j == n_load - 1) tc_commit_if(leader, &bars[B_ODONE + 1]);
+        if (next_k) {
+          issue_s(1, (gj + 1) & 1);
+          tc_commit_if(leader, &bars[B_KEMPTY + ((gj + 1) & 1)]);
+          // that was the item's last MMA reading Q: the next item's Q may land once it is done
+          if (j + 2 == n_load) tc_commit_if(leader, &bars[B_QEMPTY]);
+        }
       }
+      if (!ok) break;
+      if (n_load == 1) tc_commit_if(leader, &bars[B_QEMPTY]);
+      g = g0 + n_load;
     }
+  }
   } else {
+    reg_alloc<kRegsSoftmax>();
     // -------------------------------------------------- softmax warps 0-7
     const int t = warp >> 2;                            // query tile of this group
     const int row = (warp & 3) * 32 + lane;             // TMEM lane == query row in the tile
@@ -497,25 +610,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         m = m_new;
       }
       const float neg_mu = (m == -INFINITY) ? 0.f : -m;
-      float ls4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < kBN; c += 16) {
-        uint32_t pk[8];
-#pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          const float p0 = ex2(fmaf(s[c + e], p.scale_log2, neg_mu));
-          const float p1 = ex2(fmaf(s[c + e + 1], p.scale_log2, neg_mu));
-          ls4[(e >> 1) & 3] += p0 + p1;
-          pk[e / 2] = pack_bf16x2(p0, p1);
-        }
-        tmem_st8(s_addr + c / 2, pk);           // P row over the consumed S columns
-      }
-      const float ls = (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
-      l = l * alpha + ls;
       if constexpr (!kDenseKv<KV>) {
         // V rows of keys >= L: any bytes (cache) or never loaded (paged); the PV MMA
-        // would multiply them by p = 0.  The group that consumes the tile last zeroes
-        // them before its P arrives: tile A for j < n_kv0 (PV_A(j) is issued before
+        // would multiply them by p = 0.  The group whose PV reads the tile first zeroes
+        // them before it publishes any P: tile A for j < n_kv0 (PV_A(j) is issued before
         // PV_B(j)), tile B for the tiles only it reads.
         const int valid = itm.L - key0;
         if (valid < kBN && (warp & 3) == 0 && (t == 0 || j >= itm.n_kv0)) {
@@ -530,18 +628,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // O_t is stable here (PV_t(j-1) completed before S_t(j) did) and PV_t(j)
-      // waits for this group's arrival below
+      // waits for this group's first arrival below
+      // (16 columns at a time: the scores still occupy 128 registers)
       if (warp_raise && j > 0) {
-#pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t r[32];
-          tmem_ld32(o_addr + c, r);
+#pragma unroll 1
+        for (int c = 0; c < D; c += 16) {
+          uint32_t r[16];
+          tmem_ld16(o_addr + c, r);
           tc_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          tmem_st32(o_addr + c, r);
+          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tmem_st16(o_addr + c, r);
         }
       }
+      // p = 2^(s*scale_log2 - m), bf16 P over the consumed S columns, in two halves of 64
+      // keys: the first half is published (with the rescaled O) before the second is computed
+      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(neg_mu, neg_mu);
+      float2 sum2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      // rows with masked keys (-inf scores) take every exponential on the SFU
+      constexpr unsigned kFma = exp_fma_pairs<D>();
+      const bool soft = kFma != 0 && !__any_sync(0xffffffffu, lim < kBN);
+      if (soft) exp_store_half<0, true, kFma>(s, sc2, nm2, sum2, s_addr);
+      else exp_store_half<0, false, kFma>(s, sc2, nm2, sum2, s_addr);
+      tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[B_PHALF + t]);
+      if (soft) exp_store_half<1, true, kFma>(s, sc2, nm2, sum2, s_addr);
+      else exp_store_half<1, false, kFma>(s, sc2, nm2, sum2, s_addr);
+      const float2 sa = __fadd2_rn(sum2[0], sum2[1]), sb = __fadd2_rn(sum2[2], sum2[3]);
+      const float2 sab = __fadd2_rn(sa, sb);
+      l = l * alpha + (sab.x + sab.y);
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -597,9 +714,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (*abort_flag && warp == 9 && lane == 0) {
+  if (*abort_flag && warp == 9) {
     // a wait gave up: let every tensor-core op this CTA issued drain before TMEM is released
-    tc_commit(&bars[B_DRAIN]);
+    // (the commit comes from the lane that issued the MMAs)
+    const uint32_t leader = elect_one();
+    tc_commit_if(leader, &bars[B_DRAIN]);
     mbar_wait(&bars[B_DRAIN], 0);
   }
   __syncthreads();
@@ -685,6 +804,12 @@ cudaError_t run_prefill(const PrefillLaunch& a, cudaStream_t stream) {
   auto kern = prefill_kernel<D, KV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
+  // the softmax warpgroups' register increase waits until the producer warpgroup's
+  // decrease has made room, out of what the block was launched with: refuse a build
+  // whose launch register count could not cover the split
+  cudaFuncAttributes fa;
+  if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
+  if (fa.numRegs * kThreads < 2 * 128 * kRegsSoftmax + 128 * kRegsIo) return cudaErrorInvalidConfiguration;
   // persistent: one CTA per SM (each owns all 512 TMEM columns)
   int dev = 0, sms = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
