@@ -16,6 +16,13 @@ device time.  Both are whole-job figures: summed over ranks, divided by the
 slowest rank's time.  Inputs (192 MiB prefill, 1 GB cache) exceed the 126 MB
 L2, so no explicit flush is needed.
 
+The default run then times every configuration alone -- the oracle-sized causal
+prefill (B1 Hq4 Hkv2 N256 d64), the GPT-2-small prefill (B8 H12 N1024 d64),
+the Llama-3.1-8B causal N=4096 and non-causal N=8192 prefills, the contiguous
+decode and the paged decode with 1 and 4 new tokens -- each with its own
+roofline object under ``configs`` and its own clock record (L2 flushed before
+each launch where the inputs fit in L2).
+
 ``--impl reference`` times the fp64 CPU oracle on bounded samples of the same
 workload instead (rank 0 only).  ``--workload`` selects another shape set for
 manual runs; the default is the one described above.
@@ -331,6 +338,26 @@ def run_ours(args, world, rank, local):
     dec_gbs = tot_bytes / (dec_max * 1e-3) / 1e9
     dec_tflops = tot_dflops / (dec_max * 1e-3) / 1e12
 
+    # -------- every configuration alone (the default run only), inside the clock record
+    configs = None
+    if args.workload == DEFAULT_SET and not args.no_configs:
+        peaks0, src0 = load_peaks()
+        clocks2 = ClockSampler(local)
+        clocks2.start()
+        time.sleep(0.3)
+        if world > 1:
+            dist.barrier()
+        c0 = time.time()
+        configs = run_configs(kv, torch, dev, stream, args, world, peaks0, src0)
+        c1 = time.time()
+        clocks2.window = (c0, c1)
+        time.sleep(0.25)
+        clocks2.stop()
+        configs["clocks"] = clocks2.summary()
+        status = kv.attn_get_device_status(clear=True)
+        if status != 0:
+            raise RuntimeError(f"device status {status} during the configuration runs")
+
     # -------- end to end through the public API with host buffers (pinned)
     e2e = None if args.no_e2e else run_e2e(kv, torch, dev, stream, wp, wd, q, k, v, case, table, msk, ws, args,
                                            world, scales, prefill_cache)
@@ -384,15 +411,112 @@ def run_ours(args, world, rank, local):
             "decode": {"value": round(dec_gbs, 1), "unit": "GB/s", "tflops": round(dec_tflops, 2),
                        "roofline": roof_dec, "append_ms_per_step": round(ap_ms / K, 4)},
             "roofline": roof_pf,
+            "configs": configs,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            # per step: prefill, append, then decode split + combine (or one attn_prefill_cache launch)
+            # per step: prefill, append, then decode split + combine (or one attn_prefill_cache launch);
+            # the configuration runs are outside the timed region
             "gpu_launches": (3 if prefill_cache else 4) * K,
             "clocks": clocks.summary(),
         }
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+    return out
+
+
+# Every configuration the method is specified on, timed in the default run after the step
+# (name, workload, note).  Configuration 1 is the oracle-sized parity case.
+CONFIG_RUNS = [
+    ("1_prefill_small", "prefill_small", "parity-size case (the oracle's full-output case); L2 flushed before each launch"),
+    ("2_prefill_gpt2", "prefill_gpt2", "GPT-2-small MHA; inputs fit in L2, so L2 is flushed before each launch"),
+    ("3_prefill_llama8b_causal", "prefill_llama8b", "inputs larger than L2"),
+    ("3_prefill_llama8b_noncausal_8192", "prefill_llama8b_nc", "inputs larger than L2"),
+    ("4_decode_contig_t1", "decode_contig", "kv_append then attn_decode; cache larger than L2"),
+    ("5_decode_paged_t1", "decode_paged", "kv_append then attn_decode; cache larger than L2"),
+    ("5_decode_paged_t4", "decode_paged_t4", "speculative-verify shape, offset mask; cache larger than L2"),
+]
+L2_FLUSH_BYTES = 256 << 20   # twice the 126 MB L2
+
+
+def run_configs(kv, torch, dev, stream, args, world, peaks, peak_src):
+    """Each configuration alone: warm-up launches, then n timed launches, CUDA events
+    around the kernel call only (an L2 flush, where the inputs fit in L2, runs between
+    the events of consecutive launches).  Whole-job: units summed over ranks over the
+    slowest rank's summed time."""
+    import synth
+    n = max(5, min(args.steps, 50))
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    out = {}
+    for key, name, note in CONFIG_RUNS:
+        w = synth.WORKLOADS[name]
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        small = False
+        if isinstance(w, synth.Prefill):
+            q, k, v = synth.prefill_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, synth.SEEDS[name], dev)
+            o = torch.empty(w.B, w.N, w.Hq, w.d, dtype=torch.bfloat16, device=dev)
+            lse = torch.empty(w.B, w.Hq, w.N, dtype=torch.float32, device=dev)
+            small = 4 * q.numel() * 2 < 126e6
+
+            def call():
+                kv.attn_prefill(q, k, v, o, lse, scale=w.scale, causal=w.causal, stream=stream)
+            units, unit_name = prefill_flops(w), "flops"
+            kernel = f"prefill_kernel<{w.d}>"
+        else:
+            case = synth.decode_inputs(w.B, w.T, w.Hq, w.Hkv, w.d, w.len_lo, w.len_hi, synth.SEEDS[name], device=dev,
+                                       paged=w.paged, fp8=w.fp8)
+            cl = torch.as_tensor(case.cache_lens.astype(np.int32), device=dev)
+            sl = torch.as_tensor(case.seqlens_k.astype(np.int32), device=dev)
+            tab = None if case.page_table is None else torch.as_tensor(case.page_table, device=dev)
+            kc = case.k_pool if w.paged else case.k_cache
+            vc = case.v_pool if w.paged else case.v_cache
+            msk = int(case.seqlens_k.max())
+            od = torch.empty(w.B, w.T, w.Hq, w.d, dtype=torch.bfloat16, device=dev)
+            ld = torch.empty(w.B, w.Hq, w.T, dtype=torch.float32, device=dev)
+            ws = kv.decode_workspace(w.B, w.T, w.Hq, w.Hkv, w.d, msk, 0, dev)
+            kv.kv_append(kc, vc, case.k_new, case.v_new, cl, page_table=tab, stream=stream)
+
+            def call():
+                kv.attn_decode(case.q, kc, vc, sl, od, ld, page_table=tab, max_seqlen_k=msk, scale=w.scale,
+                               causal=w.causal, workspace=ws, stream=stream)
+            units, unit_name = decode_bytes(case, w), "bytes"
+            kernel = decode_kernel_name(w)
+        for _ in range(3):
+            call()
+        for i in range(n):
+            if small:
+                flush.fill_(float(i))
+            ev[i][0].record(stream)
+            call()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        ms = sum(a.elapsed_time(b) for a, b in ev)
+        tot, ms_max = reduce_over_ranks(units * n, ms, world, dev)
+        per_launch = units / (ms / n * 1e-3)
+        if unit_name == "flops":
+            value, unit = tot / (ms_max * 1e-3) / 1e12, "TFLOP/s"
+            roof = {"bound": "tensor", "achieved": round(per_launch / 1e12, 1), "peak": peaks["bf16_tflops"],
+                    "unit": "TFLOP/s", "frac": round(per_launch / 1e12 / peaks["bf16_tflops"], 4),
+                    "frac_of_sustained": round(per_launch / 1e12 / peaks["bf16_tflops_sustained"], 4),
+                    "peak_source": f"{peak_src} (bf16 burst)", "flops_per_launch": units}
+        else:
+            value, unit = tot / (ms_max * 1e-3) / 1e9, "GB/s"
+            roof = {"bound": "hbm", "achieved": round(per_launch / 1e9, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(per_launch / 1e9 / peaks["hbm_gbs"], 4), "peak_source": f"{peak_src} (copy)",
+                    "bytes_per_launch": units}
+        roof["kernel"] = kernel
+        roof["launch_ms"] = round(ms / n, 4)
+        desc = {"B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d}
+        if isinstance(w, synth.Prefill):
+            desc.update(N=w.N, causal=w.causal, o_dtype="bf16")
+        else:
+            desc.update(T=w.T, cache_len=[w.len_lo, w.len_hi], paged=w.paged, o_dtype="bf16")
+        out[key] = {"workload": name, "shape": desc, "value": round(value, 2), "unit": unit, "launches": n,
+                    "note": note, "roofline": roof}
+        del call
+        torch.cuda.synchronize(dev)
+    del flush
+    torch.cuda.empty_cache()
     return out
 
 
@@ -672,6 +796,7 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration runs")
     ap.add_argument("--ref-step-budget", type=float, default=1.5, help="seconds of oracle work per reference step")
     args = ap.parse_args(argv)
     if args.warmup < 3:
