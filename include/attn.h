@@ -296,10 +296,17 @@ ATTN_API int attn_selftest_wait_timeout(void* stream);
  *     Nothing in it has to start at zero (every partial is written before it is
  *     read), but calls whose kernels overlap on the GPU -- on different streams,
  *     or from different host threads -- race on it: serialise them.
- *   - Returns ATTN_ERR_WORKSPACE, before launching anything, when the request
- *     needs more than ATTN_DECODE_NOALLOC_SCRATCH_BYTES of partials (the figure
- *     attn_decode_workspace_bytes reports); a smaller num_splits needs less.
- *     Every other error is attn_decode's.
+ *   - The request is checked exactly as attn_decode checks it, with a
+ *     workspace of ATTN_DECODE_NOALLOC_SCRATCH_BYTES: argument errors come
+ *     first, with attn_decode's codes; then ATTN_ERR_WORKSPACE, before anything
+ *     is launched, when this request's own partials do not fit in the array
+ *     (attn_decode_workspace_bytes reports the larger of the bf16 and FP8
+ *     layouts, so it can exceed what this call needs); a smaller num_splits
+ *     needs less.
+ *   - The array's device address is looked up once per device and kept for the
+ *     life of the process; like the library's status word and work-queue
+ *     counters it does not survive cudaDeviceReset or the destruction of the
+ *     device's primary context.
  */
 #define ATTN_DECODE_NOALLOC_SCRATCH_BYTES (32u << 20) /* 32 MiB */
 

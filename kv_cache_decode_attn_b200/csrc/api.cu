@@ -194,7 +194,7 @@ int decode_impl(const void* q, const void* k_cache, const void* v_cache, const f
                 bool fp8, const int32_t* seqlens_k, const int32_t* page_table, int max_blocks_per_seq,
                 int num_blocks, int cache_capacity, int max_seqlen_k, void* o, int o_dtype, float* lse, int B, int T,
                 int Hq, int Hkv, int d, float scale, int causal, int num_splits, void* workspace,
-                size_t workspace_bytes, void* stream, const char* name) {
+                size_t workspace_bytes, void* stream, const char* name, bool static_scratch = false) {
   if (!q || !k_cache || !v_cache || !seqlens_k || !o) return ATTN_ERR_INVALID_ARG;
   if (fp8 && (!k_scale || !v_scale)) return ATTN_ERR_INVALID_ARG;
   if (B < 1 || T < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || num_splits < 0) return ATTN_ERR_INVALID_ARG;
@@ -220,7 +220,13 @@ int decode_impl(const void* q, const void* k_cache, const void* v_cache, const f
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
   DecodeLayout L;
   if (!decode_layout(B, T, Hq, Hkv, d, max_seqlen_k, num_splits, fp8, &L)) return ATTN_ERR_INVALID_ARG;
-  if (!workspace || workspace_bytes < L.total || !aligned16(workspace)) return ATTN_ERR_WORKSPACE;
+  if (workspace_bytes < L.total) return ATTN_ERR_WORKSPACE;
+  if (static_scratch) {
+    // attn_decode_noalloc: the library's own array, looked up only once the request is known to be valid
+    workspace = noalloc_scratch();
+    if (!workspace) return ATTN_ERR_CUDA;
+  }
+  if (!workspace || !aligned16(workspace)) return ATTN_ERR_WORKSPACE;
   unsigned* st = status_ptr();
   if (!st) return ATTN_ERR_CUDA;
   DecodeLaunch a;
@@ -347,6 +353,15 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
   return decode_impl(q, k_cache, v_cache, nullptr, nullptr, false, seqlens_k, page_table, max_blocks_per_seq,
                      num_blocks, cache_capacity, max_seqlen_k, o, o_dtype, lse, B, T, Hq, Hkv, d, scale, causal,
                      num_splits, workspace, workspace_bytes, stream, "attn_decode");
+}
+
+int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens_k,
+                        const int32_t* page_table, int max_blocks_per_seq, int num_blocks, int cache_capacity,
+                        int max_seqlen_k, void* o, int o_dtype, float* lse, int B, int T, int Hq, int Hkv, int d,
+                        float scale, int causal, int num_splits, void* stream) {
+  return decode_impl(q, k_cache, v_cache, nullptr, nullptr, false, seqlens_k, page_table, max_blocks_per_seq,
+                     num_blocks, cache_capacity, max_seqlen_k, o, o_dtype, lse, B, T, Hq, Hkv, d, scale, causal,
+                     num_splits, nullptr, ATTN_DECODE_NOALLOC_SCRATCH_BYTES, stream, "attn_decode_noalloc", true);
 }
 
 int attn_decode_fp8(const void* q, const void* k_cache, const void* v_cache, const float* k_scale,

@@ -1,6 +1,7 @@
-// attn_decode_noalloc: attn_decode with its partials in a file-scope device
-// array instead of a caller-provided workspace, for callers that cannot
-// allocate device memory (see include/attn.h).
+// The static device array behind attn_decode_noalloc: decode partials for callers
+// that cannot allocate device memory (include/attn.h says who they are).  The entry
+// point itself is in api.cu; it validates the request exactly as attn_decode does and
+// only then asks for this array.
 #include <mutex>
 
 #include "../../include/attn.h"
@@ -13,10 +14,15 @@ static __device__ __align__(256) unsigned char g_decode_scratch[ATTN_DECODE_NOAL
 
 constexpr int kMaxDevices = 64;
 
+}  // namespace
+
+namespace kvattn {
+
 // Device address of g_decode_scratch on the current device, looked up once per
 // device with that device current.  In host code the array's name is only a
-// host-side stand-in: passing it to a kernel would read the wrong memory.
-void* scratch_on_current_device() {
+// host-side stand-in: passing it to a kernel would read the wrong memory.  The
+// address is kept for the life of the process (a context reset invalidates it).
+void* noalloc_scratch() {
   static void* ptrs[kMaxDevices] = {};
   static std::mutex mu;
   int dev = 0;
@@ -30,27 +36,4 @@ void* scratch_on_current_device() {
   return ptrs[dev];
 }
 
-}  // namespace
-
-extern "C" ATTN_API int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
-                                            const int32_t* seqlens_k, const int32_t* page_table,
-                                            int max_blocks_per_seq, int num_blocks, int cache_capacity,
-                                            int max_seqlen_k, void* o, int o_dtype, float* lse, int B, int T,
-                                            int Hq, int Hkv, int d, float scale, int causal, int num_splits,
-                                            void* stream) {
-  // the key-length bound attn_decode will use (0 means the cache capacity)
-  long long bound = max_seqlen_k;
-  if (bound == 0) bound = page_table ? (long long)max_blocks_per_seq * kvattn::kPageTokens : cache_capacity;
-  if (bound > 0 && bound <= INT32_MAX) {
-    const size_t need = attn_decode_workspace_bytes(B, T, Hq, Hkv, d, (int)bound, num_splits);
-    if (need > ATTN_DECODE_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_WORKSPACE;
-  }
-  void* scratch = nullptr;
-  if (q && k_cache && v_cache && seqlens_k && o) {   // argument errors are reported by attn_decode itself
-    scratch = scratch_on_current_device();
-    if (!scratch) return ATTN_ERR_CUDA;
-  }
-  return attn_decode(q, k_cache, v_cache, seqlens_k, page_table, max_blocks_per_seq, num_blocks, cache_capacity,
-                     max_seqlen_k, o, o_dtype, lse, B, T, Hq, Hkv, d, scale, causal, num_splits, scratch,
-                     ATTN_DECODE_NOALLOC_SCRATCH_BYTES, stream);
-}
+}  // namespace kvattn

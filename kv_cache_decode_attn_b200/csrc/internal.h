@@ -107,6 +107,10 @@ int encode_tmap_3d(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t d
                    uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1, uint32_t box2,
                    int elem_bytes = 2);
 
+// Device address, on the current device, of the static array attn_decode_noalloc keeps
+// its partials in (ATTN_DECODE_NOALLOC_SCRATCH_BYTES), or nullptr if it cannot be had.
+void* noalloc_scratch();
+
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream);
 // tcgen05 split kernel for more than 16 query rows per KV head (K/V maps with 128-row boxes when contiguous)
 cudaError_t launch_decode_tc(const DecodeLaunch& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream);
