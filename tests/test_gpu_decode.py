@@ -280,12 +280,17 @@ def test_append_out_of_range_sets_status():
 
 
 # ----------------------------------------------------- full-size workloads
-def _sampled_rows_check(name, n_rows=12, seed=0):
+def _sampled_rows_check(name, n_rows=12, seed=0, whole_groups=(), o_dtype=torch.float32):
+    """Random (sequence, query head) picks, plus every query head of the (sequence,
+    KV head) groups in whole_groups (negative indices count from the end)."""
     w, case = synth.workload_decode(name, device="cuda")
     T, Hq, Hkv, d, G = w.T, w.Hq, w.Hkv, w.d, w.Hq // w.Hkv
     # host copies of what the oracle needs, taken before the append
     rng = np.random.default_rng(seed)
     picks = [(int(rng.integers(w.B)), int(rng.integers(Hq))) for _ in range(n_rows)]
+    for b, g in whole_groups:
+        b, g = b % w.B, g % Hkv
+        picks += [(b, g * G + j) for j in range(G)]
     needed = {}
     for b, h in picks:
         g = h // G
@@ -299,7 +304,7 @@ def _sampled_rows_check(name, n_rows=12, seed=0):
         else:
             needed[(b, g)] = (case.k_cache[b, :L0, g].cpu(), case.v_cache[b, :L0, g].cpu(), None)
     q_h, kn_h, vn_h = case.q.cpu(), case.k_new.cpu(), case.v_new.cpu()
-    o, lse = run_step(case, T, Hq, Hkv, d, w.scale, max_seqlen_k=int(case.seqlens_k.max()))
+    o, lse = run_step(case, T, Hq, Hkv, d, w.scale, max_seqlen_k=int(case.seqlens_k.max()), o_dtype=o_dtype)
     torch.cuda.synchronize()
     for b, h in picks:
         g = h // G
@@ -323,4 +328,11 @@ def _sampled_rows_check(name, n_rows=12, seed=0):
 @pytest.mark.parametrize("name", ["decode_contig", "decode_paged", "decode_paged_t4", "decode_paged_t8"])
 def test_full_size_workload_sampled_rows(name):
     _sampled_rows_check(name)
+    torch.cuda.empty_cache()
+
+
+def test_full_size_paged_t4_whole_groups_bf16_output():
+    """The T=4 paged workload with bf16 O: every query head and token of the first
+    and the last (sequence, KV head) group, plus random picks."""
+    _sampled_rows_check("decode_paged_t4", n_rows=8, seed=3, whole_groups=[(0, 0), (-1, -1)], o_dtype=torch.bfloat16)
     torch.cuda.empty_cache()

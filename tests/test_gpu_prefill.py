@@ -135,6 +135,33 @@ def test_prefill_llama_workload_sampled_rows(name):
     torch.cuda.empty_cache()
 
 
+@pytest.mark.parametrize("name", ["prefill_llama8b", "prefill_llama8b_nc"])
+def test_prefill_llama_workload_whole_heads_bf16_output(name):
+    """The Llama workloads as the benchmark runs them (bf16 O): every row of two
+    whole (b, h) heads -- the first head of the first sequence (K/V head 0) and the
+    last head of the last sequence (the last K/V head) -- against the oracle's own
+    attention over that head, its mask included."""
+    w, (q, k, v) = synth.workload_prefill(name, device="cuda")
+    o, lse = run_prefill(q, k, v, w.scale, w.causal, o_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    G = w.Hq // w.Hkv
+    for b, h in [(0, 0), (w.B - 1, w.Hq - 1)]:
+        g = oracle.kv_head_for(h, w.Hq, w.Hkv)
+        assert g == h // G
+        K, V = f64(k[b, :, g]), f64(v[b, :, g])
+        # rows in blocks (exact for any mask: each row's softmax is its own)
+        rows = 1024 if w.causal else 512
+        for i0 in range(0, w.N, rows):
+            i1 = min(w.N, i0 + rows)
+            nk = i1 if w.causal else w.N     # causal: rows i0..i1-1 are the last rows of the first i1 keys
+            o_ref, lse_ref = oracle.attention(f64(q[b:b + 1, i0:i1, h:h + 1]), K[None, :nk, None],
+                                              V[None, :nk, None], w.scale, w.causal)
+            check_o(o[b:b + 1, i0:i1, h:h + 1], o_ref, f"{name} b={b} h={h} rows {i0}..{i1 - 1}")
+            check_lse(lse[b:b + 1, h:h + 1, i0:i1], lse_ref, f"{name} b={b} h={h} rows {i0}..{i1 - 1}")
+    del q, k, v, o, lse
+    torch.cuda.empty_cache()
+
+
 @pytest.mark.parametrize("B,Hq,Hkv,N,d,causal", [
     (2, 4, 2, 8200, 128, True),     # long sequences: items grouped by K/V head, ragged last block
     (1, 4, 1, 16400, 64, True),
