@@ -85,6 +85,10 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsIo <= 168 * kThreads, "registe
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 of the largest allowed p
+// K/V ring depth (a third K stage, which fits at d = 128, measured no faster: the
+// copies are issued about one KV step ahead of their use).
+constexpr int kKStages = 2;
+constexpr int kVStages = 2;
 
 template <int D>
 struct PrefillCfg {
@@ -92,14 +96,15 @@ struct PrefillCfg {
   static constexpr int kTileBytes = kBN * D * 2;          // one Q, K or V tile
   static constexpr int kHalfBytes = kBN * 128;            // 128 rows x 128 B
   static constexpr int kQOff = 0;                         // Q_A, Q_B
-  static constexpr int kKOff = kQOff + 2 * kTileBytes;    // K stages 0, 1
-  static constexpr int kVOff = kKOff + 2 * kTileBytes;    // V stages 0, 1
-  static constexpr int kBarOff = kVOff + 2 * kTileBytes;
+  static constexpr int kKOff = kQOff + 2 * kTileBytes;          // K stages 0..kKStages-1
+  static constexpr int kVOff = kKOff + kKStages * kTileBytes;   // V stages 0, 1
+  static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
   static constexpr int kOrderOff = kBarOff + 256;        // cached forms: sequences by length, longest first
   static constexpr int kMaxOrdered = 256;
   static constexpr int kUsed = kOrderOff + kMaxOrdered * 4;
   // one CTA per SM: it owns all 512 TMEM columns
   static constexpr int kSmemBytes = (kUsed + 1024) > 120 * 1024 ? (kUsed + 1024) : 120 * 1024;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory of one CTA");
   static constexpr int kTmemCols = 512;
   // TMEM columns: S of tile t at 128*t, O of tile t at 256 + D*t
   __host__ __device__ static constexpr int s_col(int t) { return 128 * t; }
@@ -108,19 +113,20 @@ struct PrefillCfg {
 
 enum Bar {
   B_QFULL = 0,
-  B_QEMPTY = 1,   // all MMAs of an item done: its Q tiles may be replaced
-  B_KFULL = 2,    // +stage
-  B_VFULL = 4,    // +stage
-  B_KEMPTY = 6,   // +stage: both S MMAs reading this K stage are done
-  B_VEMPTY = 8,   // +stage: both PV MMAs reading this V stage are done
-  B_SFULL = 10,   // +tile
-  B_PHALF = 12,   // +tile: P of the tile's first 64 keys is in TMEM (and O is rescaled)
-  B_PFULL = 14,   // +tile: P of all 128 keys is in TMEM
-  B_ODONE = 16,   // +tile: last PV of an item done
-  B_OFREE = 18,   // +tile: the softmax group has read O out
-  B_DRAIN = 20,   // only used when a bounded wait gave up
-  B_COUNT = 21
+  B_QEMPTY = 1,                     // all MMAs of an item done: its Q tiles may be replaced
+  B_KFULL = 2,                      // +K stage
+  B_KEMPTY = B_KFULL + kKStages,    // +K stage: both S MMAs reading this K stage are done
+  B_VFULL = B_KEMPTY + kKStages,    // +V stage
+  B_VEMPTY = B_VFULL + kVStages,    // +V stage: both PV MMAs reading this V stage are done
+  B_SFULL = B_VEMPTY + kVStages,    // +tile
+  B_PHALF = B_SFULL + 2,            // +tile: P of the tile's first 64 keys is in TMEM (and O is rescaled)
+  B_PFULL = B_PHALF + 2,            // +tile: P of all 128 keys is in TMEM
+  B_ODONE = B_PFULL + 2,            // +tile: last PV of an item done
+  B_OFREE = B_ODONE + 2,            // +tile: the softmax group has read O out
+  B_DRAIN = B_OFREE + 2,            // only used when a bounded wait gave up
+  B_COUNT = B_DRAIN + 1
 };
+static_assert(B_COUNT * 8 + 16 <= 256, "barrier block");
 
 // Where K and V come from.
 // KV_DENSE_GROUPED: the dense form with its items in the cached forms' order.
@@ -249,6 +255,7 @@ constexpr unsigned exp_fma_pairs() { return D == 64 ? 0x92u : 0u; }
 template <int HALF, bool FMA, unsigned kExpFmaPairs>
 __device__ __forceinline__ void exp_store_half(const float (&s)[kBN], float2 sc, float2 nm, float2 (&sum2)[4],
                                                uint32_t taddr) {
+  // one TMEM store per 16 keys (measured faster than stores of 32 or 64 keys)
 #pragma unroll
   for (int c = HALF * (kBN / 2); c < (HALF + 1) * (kBN / 2); c += 16) {
     uint32_t pk[8];
@@ -298,11 +305,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(&bars[B_QFULL], 1);
     mbar_init(&bars[B_QEMPTY], 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(&bars[B_KFULL + s], 1);
-      mbar_init(&bars[B_VFULL + s], 1);
       mbar_init(&bars[B_KEMPTY + s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(&bars[B_VFULL + s], 1);
       mbar_init(&bars[B_VEMPTY + s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[B_SFULL + s], 1);
       mbar_init(&bars[B_PHALF + s], 4);
       mbar_init(&bars[B_PFULL + s], 4);
@@ -332,7 +343,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t keep = policy_evict_last();    // K/V tiles are re-read by other query blocks and heads
       const uint64_t once = policy_evict_first();
       int g = 0, it = 0, q_loaded = 0;              // K/V tiles loaded, items started, Q loads issued
-      int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};   // last K / V tile whose copy was issued per stage
+      int last_k[kKStages], last_v[kVStages];   // last K / V tile whose copy was issued per stage
+#pragma unroll
+      for (int i = 0; i < kKStages; ++i) last_k[i] = -1;
+#pragma unroll
+      for (int i = 0; i < kVStages; ++i) last_v[i] = -1;
       bool ok = true, clean_end = false;
       for (int w = blockIdx.x;; ++it) {
         // Q of the previous item no longer read (this also means its copy landed)
@@ -376,29 +391,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         if constexpr (KV == KV_PAGED) read_ids(0);
         for (int t = 0; t < itm.n_load; ++t, ++g) {
-          const int st = g & 1;
-          // K of this stage is released after the second S MMA reading it, V after the
-          // second PV MMA, so the next K tile lands while the current PVs still run
-          if (g >= 2 && !wait_or_abort(&bars[B_KEMPTY + st], ((g >> 1) - 1) & 1, abort_flag, p.status)) {
+          const int ks = g % kKStages, vs = g % kVStages;
+          // K of a stage is released after the second S MMA reading it, V after the
+          // second PV MMA, so the next K tiles land while the current PVs still run
+          if (g >= kKStages &&
+              !wait_or_abort(&bars[B_KEMPTY + ks], ((g / kKStages) - 1) & 1, abort_flag, p.status)) {
             ok = false;
             break;
           }
-          last_k[st] = g;
+          last_k[ks] = g;
           if constexpr (KV != KV_PAGED) {
-            mbar_arrive_expect_tx(&bars[B_KFULL + st], C::kTileBytes);
+            mbar_arrive_expect_tx(&bars[B_KFULL + ks], C::kTileBytes);
 #pragma unroll
             for (int hh = 0; hh < C::kHalves; ++hh)
-              tma_load_4d(smem + C::kKOff + st * C::kTileBytes + hh * C::kHalfBytes, &tmK, &bars[B_KFULL + st],
+              tma_load_4d(smem + C::kKOff + ks * C::kTileBytes + hh * C::kHalfBytes, &tmK, &bars[B_KFULL + ks],
                           hh * 64, kvh, t * kBN, itm.b, keep);
-            if (g >= 2 && !wait_or_abort(&bars[B_VEMPTY + st], ((g >> 1) - 1) & 1, abort_flag, p.status)) {
+            if (g >= kVStages &&
+                !wait_or_abort(&bars[B_VEMPTY + vs], ((g / kVStages) - 1) & 1, abort_flag, p.status)) {
               ok = false;
               break;
             }
-            last_v[st] = g;
-            mbar_arrive_expect_tx(&bars[B_VFULL + st], C::kTileBytes);
+            last_v[vs] = g;
+            mbar_arrive_expect_tx(&bars[B_VFULL + vs], C::kTileBytes);
 #pragma unroll
             for (int hh = 0; hh < C::kHalves; ++hh)
-              tma_load_4d(smem + C::kVOff + st * C::kTileBytes + hh * C::kHalfBytes, &tmV, &bars[B_VFULL + st],
+              tma_load_4d(smem + C::kVOff + vs * C::kTileBytes + hh * C::kHalfBytes, &tmV, &bars[B_VFULL + vs],
                           hh * 64, kvh, t * kBN, itm.b, keep);
           } else {
             // one 16-row box per physical block holding keys of this tile below L
@@ -410,28 +427,29 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
             const uint32_t bytes = nb * C::kHalves * kPageTokens * 128;
-            mbar_arrive_expect_tx(&bars[B_KFULL + st], bytes);
+            mbar_arrive_expect_tx(&bars[B_KFULL + ks], bytes);
 #pragma unroll
             for (int jb = 0; jb < kBlocks; ++jb) {
               if (jb >= nb) break;
 #pragma unroll
               for (int hh = 0; hh < C::kHalves; ++hh)
-                tma_load_3d(smem + C::kKOff + st * C::kTileBytes + hh * C::kHalfBytes + jb * kPageTokens * 128, &tmK,
-                            &bars[B_KFULL + st], hh * 64, kvh, ids[jb] * kPageTokens, keep);
+                tma_load_3d(smem + C::kKOff + ks * C::kTileBytes + hh * C::kHalfBytes + jb * kPageTokens * 128, &tmK,
+                            &bars[B_KFULL + ks], hh * 64, kvh, ids[jb] * kPageTokens, keep);
             }
-            if (g >= 2 && !wait_or_abort(&bars[B_VEMPTY + st], ((g >> 1) - 1) & 1, abort_flag, p.status)) {
+            if (g >= kVStages &&
+                !wait_or_abort(&bars[B_VEMPTY + vs], ((g / kVStages) - 1) & 1, abort_flag, p.status)) {
               ok = false;
               break;
             }
-            last_v[st] = g;
-            mbar_arrive_expect_tx(&bars[B_VFULL + st], bytes);
+            last_v[vs] = g;
+            mbar_arrive_expect_tx(&bars[B_VFULL + vs], bytes);
 #pragma unroll
             for (int jb = 0; jb < kBlocks; ++jb) {
               if (jb >= nb) break;
 #pragma unroll
               for (int hh = 0; hh < C::kHalves; ++hh)
-                tma_load_3d(smem + C::kVOff + st * C::kTileBytes + hh * C::kHalfBytes + jb * kPageTokens * 128, &tmV,
-                            &bars[B_VFULL + st], hh * 64, kvh, ids[jb] * kPageTokens, keep);
+                tma_load_3d(smem + C::kVOff + vs * C::kTileBytes + hh * C::kHalfBytes + jb * kPageTokens * 128, &tmV,
+                            &bars[B_VFULL + vs], hh * 64, kvh, ids[jb] * kPageTokens, keep);
             }
             if (t + 1 < itm.n_load) read_ids(t + 1);
           }
@@ -442,10 +460,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // no copy may still be landing in shared memory when the CTA exits (after a clean
       // end, the wait on B_QEMPTY above already covered the last Q copy)
       if (!clean_end && q_loaded > 0) mbar_wait(&bars[B_QFULL], (q_loaded - 1) & 1);
-      for (int st = 0; st < 2; ++st) {
-        if (last_k[st] >= 0) mbar_wait(&bars[B_KFULL + st], (last_k[st] >> 1) & 1);
-        if (last_v[st] >= 0) mbar_wait(&bars[B_VFULL + st], (last_v[st] >> 1) & 1);
-      }
+      for (int i = 0; i < kKStages; ++i)
+        if (last_k[i] >= 0) mbar_wait(&bars[B_KFULL + i], (last_k[i] / kKStages) & 1);
+      for (int i = 0; i < kVStages; ++i)
+        if (last_v[i] >= 0) mbar_wait(&bars[B_VFULL + i], (last_v[i] / kVStages) & 1);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------- MMA issuer
@@ -462,11 +480,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // precomputed base (Q tile, K or V ring stage) plus a compile-time K-step offset
     const uint32_t sbase = smem_u32(smem);
     const uint32_t q_lo0 = desc_lo(sbase + C::kQOff, 16), q_lo1 = desc_lo(sbase + C::kQOff + C::kTileBytes, 16);
-    const uint32_t k_lo0 = desc_lo(sbase + C::kKOff, 16), k_lo1 = desc_lo(sbase + C::kKOff + C::kTileBytes, 16);
+    const uint32_t k_lo0 = desc_lo(sbase + C::kKOff, 16);
     const uint32_t v_lo0 = desc_lo(sbase + C::kVOff, C::kHalfBytes);
-    const uint32_t v_lo1 = desc_lo(sbase + C::kVOff + C::kTileBytes, C::kHalfBytes);
-    auto issue_s = [&](int t, int st) {     // S_t = Q_t K^T, K in ring stage st
-      const uint32_t qa = t ? q_lo1 : q_lo0, kb = st ? k_lo1 : k_lo0;
+    constexpr uint32_t kStageLo = C::kTileBytes >> 4;     // one ring stage in descriptor units
+    auto issue_s = [&](int t, int ks) {     // S_t = Q_t K^T, K in ring stage ks
+      const uint32_t qa = t ? q_lo1 : q_lo0, kb = k_lo0 + ks * kStageLo;
       const uint32_t d = tmem + C::s_col(t);
       tc_mma_ss_lo<0>(leader, d, qa, kb, idS);
 #pragma unroll
@@ -477,8 +495,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit_if(leader, &bars[B_SFULL + t]);
     };
     // O_t (+)= P_t V over keys 64*half .. 64*half+63; P_t sits in the first 64 columns of S_t
-    auto issue_pv = [&](int t, int st, bool first, int half) {
-      const uint32_t vb = st ? v_lo1 : v_lo0;
+    auto issue_pv = [&](int t, int vs, bool first, int half) {
+      const uint32_t vb = v_lo0 + vs * kStageLo;
       const uint32_t d = tmem + C::o_col(t), pa = tmem + C::s_col(t);
 #pragma unroll
       for (int k4 = 0; k4 < kBN / 32; ++k4) {
@@ -511,16 +529,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n_load = __shfl_sync(0xffffffffu, itm.n_load, 0);
       const int n_kv0 = __shfl_sync(0xffffffffu, itm.n_kv0, 0);
       const int g0 = g;
-      ok = wait_or_abort(&bars[B_KFULL + (g0 & 1)], (g0 >> 1) & 1, abort_flag, p.status);
+      const int ks0 = g0 % kKStages;
+      ok = wait_or_abort(&bars[B_KFULL + ks0], (g0 / kKStages) & 1, abort_flag, p.status);
       if (!ok) break;
       tc_fence_after();
-      issue_s(0, g0 & 1);
-      issue_s(1, g0 & 1);
-      tc_commit_if(leader, &bars[B_KEMPTY + (g0 & 1)]);
+      issue_s(0, ks0);
+      issue_s(1, ks0);
+      tc_commit_if(leader, &bars[B_KEMPTY + ks0]);
       for (int j = 0; j < n_load; ++j) {
-        const int gj = g0 + j, st = gj & 1;
+        const int gj = g0 + j, st = gj % kVStages;
+        const int ksn = (gj + 1) % kKStages;     // K stage of the next tile
         const bool next_k = j + 1 < n_load;
-        ok = wait_or_abort(&bars[B_VFULL + st], (gj >> 1) & 1, abort_flag, p.status);
+        ok = wait_or_abort(&bars[B_VFULL + st], (gj / kVStages) & 1, abort_flag, p.status);
         if (!ok) break;
         if (j < n_kv0) {
           ok = pv_tile(0, st, j, it);
@@ -528,18 +548,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (j == n_kv0 - 1) tc_commit_if(leader, &bars[B_ODONE + 0]);
         }
         if (next_k) {
-          ok = wait_or_abort(&bars[B_KFULL + ((gj + 1) & 1)], ((gj + 1) >> 1) & 1, abort_flag, p.status);
+          ok = wait_or_abort(&bars[B_KFULL + ksn], ((gj + 1) / kKStages) & 1, abort_flag, p.status);
           if (!ok) break;
           tc_fence_after();
-          if (j + 1 < n_kv0) issue_s(0, (gj + 1) & 1);
+          if (j + 1 < n_kv0) issue_s(0, ksn);
         }
         ok = pv_tile(1, st, j, it);
         if (!ok) break;
         tc_commit_if(leader, &bars[B_VEMPTY + st]);        // V of this stage is no longer needed
         if (j == n_load - 1) tc_commit_if(leader, &bars[B_ODONE + 1]);
         if (next_k) {
-          issue_s(1, (gj + 1) & 1);
-          tc_commit_if(leader, &bars[B_KEMPTY + ((gj + 1) & 1)]);
+          issue_s(1, ksn);
+          tc_commit_if(leader, &bars[B_KEMPTY + ksn]);
           // that was the item's last MMA reading Q: the next item's Q may land once it is done
           if (j + 2 == n_load) tc_commit_if(leader, &bars[B_QEMPTY]);
         }
@@ -617,8 +637,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // PV_B(j)), tile B for the tiles only it reads.
         const int valid = itm.L - key0;
         if (valid < kBN && (warp & 3) == 0 && (t == 0 || j >= itm.n_kv0)) {
-          const int gj = g_item + j, st = gj & 1;
-          if (!wait_or_abort(&bars[B_VFULL + st], (gj >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+          const int gj = g_item + j, st = gj % kVStages;
+          if (!wait_or_abort(&bars[B_VFULL + st], (gj / kVStages) & 1, abort_flag, p.status)) { ok = false; break; }
           uint8_t* vst = smem + C::kVOff + st * C::kTileBytes;
           for (int idx = max(valid, 0) * 8 + lane; idx < kBN * 8; idx += 32)
 #pragma unroll
