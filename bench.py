@@ -62,6 +62,8 @@ WORKLOAD_SETS = {
     "llama8b_chunked_prefill": ("prefill_llama8b", "prefill_chunk_paged"),
     # eight new tokens per decode step: the tensor-core split kernel (64 rows per KV head)
     "llama8b_paged_t8": ("prefill_llama8b", "decode_paged_t8"),
+    # the same over an FP8 cache (tensor-core kernel converting e4m3 tiles in shared memory)
+    "llama8b_paged_t8_fp8": ("prefill_llama8b", "decode_paged_t8_fp8"),
 }
 PREFILL_CACHE_SETS = {"llama8b_prefill_cache"}   # sets whose attend step is attn_prefill_cache
 DEFAULT_SET = "llama8b_layer"
@@ -236,12 +238,15 @@ def decode_kernel_name(wd, prefill_cache=False) -> str:
 def decode_kernel(wd):
     """(name, source files) of the kernel attn_decode picks for this shape: bf16 up
     to 16 query rows per KV head on warp-level MMAs, more on tcgen05; FP8 up to
-    8 rows on the transposed-product kernel, up to 32 on the split kernel."""
+    8 rows on the transposed-product kernel, up to 32 on the split kernel, more on
+    tcgen05 (e4m3 tiles converted to bf16 in shared memory)."""
     R = wd.Hq // wd.Hkv * wd.T
     if wd.fp8:
         if R <= 8:
             return "decode_fp8_st_kernel", ("decode_fp8.cu", "split.cuh", "decode.cu")
-        return "decode_split_kernel<fp8>", ("decode.cu", "split.cuh")
+        if R <= 32:
+            return "decode_split_kernel<fp8>", ("decode.cu", "split.cuh")
+        return "decode_tc_kernel<fp8>", ("decode_tc.cu", "decode.cu")
     if R <= 16:
         return "decode_split_kernel", ("decode.cu", "split.cuh")
     return "decode_tc_kernel", ("decode_tc.cu", "decode.cu")

@@ -215,7 +215,6 @@ int decode_impl(const void* q, const void* k_cache, const void* v_cache, const f
   if (max_seqlen_k < T || max_seqlen_k > capacity_tokens) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (Hq / Hkv > 128) return ATTN_ERR_UNSUPPORTED;                       // one token's heads must fit a row tile
-  if (fp8 && (Hq / Hkv) * T > kFp8MaxRows) return ATTN_ERR_UNSUPPORTED;
   if (fp8 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
   DecodeLayout L;

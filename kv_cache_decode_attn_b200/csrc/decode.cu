@@ -681,15 +681,15 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
     return cudaErrorInvalidValue;
 
   cudaError_t e;
-  if (a.fp8) {
-    // api.cu admits d == 128 and at most kFp8MaxRows rows per KV head
+  if (tc) {
+    e = launch_decode_tc(a, tk, tv, stream);   // bf16 above 16 rows per KV head, FP8 above 32
+  } else if (a.fp8) {
+    // api.cu admits FP8 caches with d == 128 only
     if (R <= 8) e = launch_decode_fp8_rows8(tk, tv, sp, a.B, paged, stream);
     else if (R <= 16) e = paged ? run_split<128, 1, true, true>(tk, tv, sp, a.B, stream)
                            : run_split<128, 1, false, true>(tk, tv, sp, a.B, stream);
     else e = paged ? run_split<128, 2, true, true>(tk, tv, sp, a.B, stream)
                    : run_split<128, 2, false, true>(tk, tv, sp, a.B, stream);
-  } else if (tc) {
-    e = launch_decode_tc(a, tk, tv, stream);
   } else if (a.d == 128) {   // at most kDecodeMmaRows (16) rows: one row group
     e = paged ? run_split<128, 1, true>(tk, tv, sp, a.B, stream) : run_split<128, 1, false>(tk, tv, sp, a.B, stream);
   } else {

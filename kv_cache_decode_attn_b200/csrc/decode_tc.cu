@@ -50,17 +50,26 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kStages = 2;    // K/V ring stages (S is double-buffered in TMEM)
 constexpr int kCtasPerSm = 2;   // shared memory and TMEM of one CTA
 
-template <int D>
+// FP8: the cache holds e4m3 codes.  The copies land in a ring of raw stages; the K
+// (V) producer warp then converts each raw tile into one f16 K (V) tile in the
+// operand layout the MMAs read (every e4m3 value is exact in f16), and the MMAs run
+// on f16 operands: Q is converted to f16 in place once per CTA (exact for bf16
+// magnitudes 2^-14 .. 65504) and P is stored as f16.
+template <int D, bool FP8 = false>
 struct TcCfg {
   static constexpr int kHalves = D / 64;
   static constexpr int kQHalfBytes = kRows * 128;            // Q: 128 rows x 128 B per 64 columns of d
   static constexpr int kHalfBytes = kTok * 128;              // K or V tile: kTok rows x 128 B
   static constexpr int kQBytes = kRows * D * 2;
-  static constexpr int kTileBytes = kTok * D * 2;            // one K or V tile
+  static constexpr int kTileBytes = kTok * D * 2;            // one 16-bit K or V tile
+  static constexpr int kRawBytes = kTok * D;                 // one e4m3 K or V tile (FP8)
+  static constexpr int kOperandStages = FP8 ? 1 : kStages;   // 16-bit tiles the MMAs read
   static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + kQBytes;              // K stages
-  static constexpr int kVOff = kKOff + kStages * kTileBytes; // V stages
-  static constexpr int kBarOff = kVOff + kStages * kTileBytes;
+  static constexpr int kKOff = kQOff + kQBytes;              // K stages (FP8: the converted K tile)
+  static constexpr int kVOff = kKOff + kOperandStages * kTileBytes;   // V stages (FP8: the converted V tile)
+  static constexpr int kRawKOff = kVOff + kOperandStages * kTileBytes;   // FP8: raw K stages
+  static constexpr int kRawVOff = kRawKOff + (FP8 ? kStages * kRawBytes : 0);
+  static constexpr int kBarOff = kRawVOff + (FP8 ? kStages * kRawBytes : 0);
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;
   static constexpr int kSCols = kTok;                        // one S buffer (fp32 scores of a tile)
   static constexpr int kOCol = 2 * kSCols;                   // S0 | S1 | O
@@ -86,10 +95,17 @@ enum TcBar {
   T_ODONE = T_PFULL + 2,
   T_OFINAL,
   T_DRAIN,
+  T_QC,        // FP8: Q is converted to f16
+  T_KCFULL,    // FP8: the converted K tile is ready
+  T_VCFULL,
+  T_KCEMPTY,   // FP8: the MMA reading the converted K tile is done
+  T_VCEMPTY,
   T_COUNT
 };
 
 struct TcParams {
+  const float* k_scale;   // FP8: [Hkv]
+  const float* v_scale;
   const int32_t* seqlens;
   const int32_t* page_table;
   float* part_o;
@@ -111,11 +127,38 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
   return false;
 }
 
-template <int D, bool PAGED>
+// Convert one raw e4m3 tile (kTok rows of D codes, 128-byte rows with the 128-byte
+// swizzle the copy applies) into the f16 operand tile (two halves of D/2 columns,
+// kTok rows of 128 bytes, same swizzle), one warp.  Called for d = 128 only: a raw
+// row of D codes is one 128-byte swizzle span.
+template <int D>
+__device__ __forceinline__ void convert_tile_e4m3(const uint8_t* raw, uint8_t* conv, int lane) {
+#pragma unroll 4
+  for (int idx = lane; idx < kTok * 8; idx += 32) {
+    const int r = idx >> 3, c = idx & 7;                  // row, 16-code chunk (d = 16c .. 16c+15)
+    const uint4 w = *reinterpret_cast<const uint4*>(raw + r * 128 + ((c ^ (r & 7)) << 4));
+    uint32_t o[8];
+    e4m3x4_to_f16x2x2(w.x, o[0], o[1]);
+    e4m3x4_to_f16x2x2(w.y, o[2], o[3]);
+    e4m3x4_to_f16x2x2(w.z, o[4], o[5]);
+    e4m3x4_to_f16x2x2(w.w, o[6], o[7]);
+    const int c0 = (c & 3) * 2;                           // first 16-byte chunk in the half's row
+    uint8_t* rowp = conv + (c >> 2) * (kTok * 128) + r * 128;
+    *reinterpret_cast<uint4*>(rowp + ((c0 ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(rowp + (((c0 + 1) ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+// bf16 pair to f16 pair, round to nearest (exact for magnitudes 2^-14 .. 65504).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t x) {
+  return pack_f16x2(__uint_as_float(x << 16), __uint_as_float(x & 0xFFFF0000u));
+}
+
+template <int D, bool PAGED, bool FP8>
 __global__ void __launch_bounds__(224, kCtasPerSm)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const TcParams p) {
-  using C = TcCfg<D>;
+  using C = TcCfg<D, FP8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
@@ -146,6 +189,19 @@ __global__ void __launch_bounds__(224, kCtasPerSm)
   }
   const int n_tiles = (tok_end - tok_begin + kTok - 1) / kTok;
   const int active_warps = (tile_rows + 31) / 32;
+  float scale_log2 = p.scale_log2, v_mul = 1.f;   // FP8: K scale in the exponent, V scale on O
+  if constexpr (FP8) {
+    const float ks = __ldg(p.k_scale + g), vs = __ldg(p.v_scale + g);
+    scale_log2 = p.scale_log2 * ks;
+    v_mul = vs;
+    if (!(ks > 0.f && ks <= 3.402823466e38f && vs > 0.f && vs <= 3.402823466e38f)) {
+      // a scale that is not a positive finite number: the whole CTA leaves before any
+      // barrier (the scales are uniform across it)
+      if (threadIdx.x == 0 && c == 0 && rt == 0) atomicOr(p.status, DEV_SCALE);
+      for (int r = threadIdx.x; r < tile_rows; r += blockDim.x) p.part_lse[row0 + r] = NAN;
+      return;
+    }
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[T_Q], 1);
@@ -162,6 +218,11 @@ __global__ void __launch_bounds__(224, kCtasPerSm)
     mbar_init(&bars[T_ODONE], 1);
     mbar_init(&bars[T_OFINAL], 1);
     mbar_init(&bars[T_DRAIN], 1);
+    mbar_init(&bars[T_QC], 1);
+    mbar_init(&bars[T_KCFULL], 1);
+    mbar_init(&bars[T_VCFULL], 1);
+    mbar_init(&bars[T_KCEMPTY], 1);
+    mbar_init(&bars[T_VCEMPTY], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -186,7 +247,94 @@ __global__ void __launch_bounds__(224, kCtasPerSm)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4 || warp == 6) {
+  if (FP8 && (warp == 4 || warp == 6)) {
+    // ------------------------------------------------ FP8 producers and converters
+    // Lane 0 copies raw e4m3 tiles into a 2-stage ring; the whole warp converts each
+    // raw tile into the one bf16 operand tile once the MMA has finished reading the
+    // previous one, then refills the raw stage it has just read.
+    const bool is_k = warp == 4;
+    const CUtensorMap* map = is_k ? &tmK : &tmV;
+    uint8_t* raw_ring = smem + (is_k ? C::kRawKOff : C::kRawVOff);
+    uint8_t* conv = smem + (is_k ? C::kKOff : C::kVOff);
+    const int full0 = is_k ? T_KFULL : T_VFULL;
+    uint64_t* cfull = &bars[is_k ? T_KCFULL : T_VCFULL];
+    uint64_t* cempty = &bars[is_k ? T_KCEMPTY : T_VCEMPTY];
+    const uint64_t pol = policy_evict_first();
+    constexpr int kBlocks = kTok / kPageTokens;
+    auto copy_tile = [&](int i) {      // lane 0 only
+      uint8_t* base = raw_ring + (i % kStages) * C::kRawBytes;
+      uint64_t* full = &bars[full0 + i % kStages];
+      const int tt = tok_begin + i * kTok;
+      if (!PAGED) {
+        mbar_arrive_expect_tx(full, C::kRawBytes);
+        tma_load_3d(base, map, full, 0, g, b * p.capacity + tt, pol);
+      } else {
+        const int nb = min(kBlocks, (tok_end - tt + kPageTokens - 1) / kPageTokens);
+        const int32_t* tab = p.page_table + (size_t)b * p.max_blocks + tt / kPageTokens;
+        int ids[kBlocks];
+#pragma unroll
+        for (int j = 0; j < kBlocks; ++j) ids[j] = j < nb ? __ldg(tab + j) : 0;
+#pragma unroll
+        for (int j = 0; j < kBlocks; ++j)
+          if (j < nb && (ids[j] < 0 || ids[j] >= p.num_blocks)) {
+            atomicOr(p.status, DEV_PAGE_ID);
+            ids[j] = 0;   // keep the byte count; the result is flagged invalid
+          }
+        mbar_arrive_expect_tx(full, nb * kPageTokens * 128);
+#pragma unroll
+        for (int j = 0; j < kBlocks; ++j)
+          if (j < nb) tma_load_3d(base + j * kPageTokens * 128, map, full, 0, g, ids[j] * kPageTokens, pol);
+      }
+    };
+    int issued = 0;
+    if (lane == 0) {
+      prefetch_tmap(map);
+      if (is_k) {
+        mbar_arrive_expect_tx(&bars[T_Q], p.TT * p.G * D * 2);
+#pragma unroll
+        for (int hh = 0; hh < C::kHalves; ++hh)
+          tma_load_4d(smem + C::kQOff + hh * C::kQHalfBytes, &tmQ, &bars[T_Q], hh * 64, g * p.G, t0, b, pol);
+      }
+      for (; issued < kStages && issued < n_tiles; ++issued) copy_tile(issued);
+    }
+    issued = __shfl_sync(0xffffffffu, issued, 0);
+    bool ok = true;
+    if (is_k) {
+      // Q to f16 in place (same element size, same layout), then published to the MMA warp
+      ok = tc_wait(&bars[T_Q], 0, abort_flag, p.status);
+      if (ok) {
+        for (int idx = lane; idx < C::kQBytes / 16; idx += 32) {
+          uint4* q = reinterpret_cast<uint4*>(smem + C::kQOff) + idx;
+          uint4 v = *q;
+          v = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
+          *q = v;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[T_QC]);
+      }
+    }
+    for (int i = 0; ok && i < n_tiles; ++i) {
+      if (!tc_wait(&bars[full0 + i % kStages], (i / kStages) & 1, abort_flag, p.status)) break;
+      if (i > 0 && !tc_wait(cempty, (i - 1) & 1, abort_flag, p.status)) break;
+      convert_tile_e4m3<D>(raw_ring + (i % kStages) * C::kRawBytes, conv, lane);
+      fence_proxy_async_smem();       // the converted tile is read by the MMAs (async proxy)
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(cfull);
+        if (i + kStages < n_tiles) {   // the raw stage just read takes the tile kStages ahead
+          copy_tile(i + kStages);
+          ++issued;
+        }
+      }
+      issued = __shfl_sync(0xffffffffu, issued, 0);
+    }
+    // no copy may still be landing in shared memory when the CTA exits
+    if (lane == 0) {
+      if (is_k) mbar_wait(&bars[T_Q], 0);
+      for (int i = max(0, issued - kStages); i < issued; ++i) mbar_wait(&bars[full0 + i % kStages], (i / kStages) & 1);
+    }
+  } else if (warp == 4 || warp == 6) {
     // ------------------------------------------------------------- TMA producers
     if (lane == 0) {
       const bool is_k = warp == 4;
@@ -260,12 +408,16 @@ __global__ void __launch_bounds__(224, kCtasPerSm)
     // The whole warp runs the loop (warp-uniform operands, descriptors as precomputed
     // low words plus compile-time offsets); one elected lane issues and commits.
     const uint32_t leader = elect_one();
-    constexpr uint32_t idS = idesc_bf16(kRows, kTok, 0, 0);
-    constexpr uint32_t idO = idesc_bf16(kRows, D, 0, 1);
+    constexpr uint32_t idS = FP8 ? idesc_f16(kRows, kTok, 0, 0) : idesc_bf16(kRows, kTok, 0, 0);
+    constexpr uint32_t idO = FP8 ? idesc_f16(kRows, D, 0, 1) : idesc_bf16(kRows, D, 0, 1);
     const uint32_t sbase = smem_u32(smem);
     const uint32_t q_lo = desc_lo(sbase + C::kQOff, 16);
+    // the K / V operand tile of key tile i: ring stage i % kStages (bf16), the one converted tile (FP8)
+    auto k_full = [&](int i) { return FP8 ? &bars[T_KCFULL] : &bars[T_KFULL + i % kStages]; };
+    auto v_full = [&](int i) { return FP8 ? &bars[T_VCFULL] : &bars[T_VFULL + i % kStages]; };
+    auto full_parity = [&](int i) -> uint32_t { return FP8 ? (i & 1) : ((i / kStages) & 1); };
     auto issue_s = [&](int i) {
-      const int sb = i & 1, ks = i % kStages;   // S buffer, K/V ring stage
+      const int sb = i & 1, ks = FP8 ? 0 : i % kStages;   // S buffer, K operand stage
       const uint32_t k_lo = desc_lo(sbase + C::kKOff + ks * C::kTileBytes, 16);
       const uint32_t d = tmem + sb * C::kSCols;
       tc_mma_ss_lo<0>(leader, d, q_lo, k_lo, idS);
@@ -276,10 +428,10 @@ __global__ void __launch_bounds__(224, kCtasPerSm)
         tc_mma_ss_lo<1>(leader, d, q_lo + q_off, k_lo + k_off, idS);
       }
       tc_commit_if(leader, &bars[T_SFULL + sb]);
-      tc_commit_if(leader, &bars[T_KEMPTY + ks]);     // K_i is read only by S_i
+      tc_commit_if(leader, FP8 ? &bars[T_KCEMPTY] : &bars[T_KEMPTY + ks]);     // K_i is read only by S_i
     };
-    bool ok = tc_wait(&bars[T_Q], 0, abort_flag, p.status) &&
-              tc_wait(&bars[T_KFULL], 0, abort_flag, p.status);
+    bool ok = tc_wait(&bars[FP8 ? T_QC : T_Q], 0, abort_flag, p.status) &&
+              tc_wait(k_full(0), 0, abort_flag, p.status);
     if (ok) {
       tc_fence_after();
       issue_s(0);
@@ -287,16 +439,32 @@ __global__ void __launch_bounds__(224, kCtasPerSm)
     for (int i = 0; ok && i < n_tiles; ++i) {
       const int sb = i & 1, ks = i % kStages;
       if (i + 1 < n_tiles) {
-        ok = tc_wait(&bars[T_KFULL + (i + 1) % kStages], ((i + 1) / kStages) & 1, abort_flag, p.status);
+        ok = tc_wait(k_full(i + 1), full_parity(i + 1), abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
         issue_s(i + 1);   // its S buffer last held P_{i-1}, whose PV was issued before
       }
       ok = tc_wait(&bars[T_PFULL + sb], (i >> 1) & 1, abort_flag, p.status) &&
-           tc_wait(&bars[T_VFULL + ks], (i / kStages) & 1, abort_flag, p.status);
+           tc_wait(v_full(i), full_parity(i), abort_flag, p.status);
       if (!ok) break;
+      // keys at or past this CTA's end may hold anything (past L: any bytes; past a row
+      // tile's last visible key in a paged cache: blocks never loaded, stale shared
+      // memory), even NaN: zero their V rows, which the PV MMA would otherwise multiply
+      // by p = 0.  This warp consumes the V tiles' phases in order, so the wait above
+      // is for exactly this tile's V (a softmax warp's parity wait could be satisfied
+      // by the tile two phases back while this one is still being written).
+      const int valid = tok_end - (tok_begin + i * kTok);
+      if (valid < kTok) {
+        uint8_t* vst = smem + C::kVOff + (FP8 ? 0 : ks) * C::kTileBytes;
+        for (int idx = max(valid, 0) * 8 + lane; idx < kTok * 8; idx += 32)
+#pragma unroll
+          for (int hh = 0; hh < C::kHalves; ++hh)
+            *reinterpret_cast<uint4*>(vst + hh * C::kHalfBytes + idx * 16) = make_uint4(0, 0, 0, 0);
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
       tc_fence_after();
-      const uint32_t v_lo = desc_lo(sbase + C::kVOff + ks * C::kTileBytes, C::kHalfBytes);
+      const uint32_t v_lo = desc_lo(sbase + C::kVOff + (FP8 ? 0 : ks) * C::kTileBytes, C::kHalfBytes);
       const uint32_t d = tmem + C::kOCol, pa = tmem + sb * C::kSCols;
       if (i == 0) tc_mma_ts_lo<0>(leader, d, pa, v_lo, idO);
       else tc_mma_ts_lo<1>(leader, d, pa, v_lo, idO);
@@ -304,7 +472,7 @@ __global__ void __launch_bounds__(224, kCtasPerSm)
       for (int kk = 1; kk < kTok / 16; ++kk)
         tc_mma_ts_lo<1>(leader, d, pa + kk * 8, v_lo + ((kk * 16 * 128) >> 4), idO);
       tc_commit_if(leader, &bars[T_ODONE]);
-      tc_commit_if(leader, &bars[T_VEMPTY + ks]);
+      tc_commit_if(leader, FP8 ? &bars[T_VCEMPTY] : &bars[T_VEMPTY + ks]);
     }
     // also on a failed wait, so that the epilogue does not wait in vain (abort_flag marks the result)
     tc_commit_if(leader, &bars[T_OFINAL]);
@@ -347,7 +515,7 @@ __global__ void __launch_bounds__(224, kCtasPerSm)
 #pragma unroll
       for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], s[kTok - 8 + k]);
       float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
-      mx *= p.scale_log2;
+      mx *= scale_log2;
       const bool warp_raise = __any_sync(0xffffffffu, mx > m + 8.f);
       float alpha = 1.f;
       if (warp_raise) {
@@ -362,10 +530,10 @@ __global__ void __launch_bounds__(224, kCtasPerSm)
         uint32_t pk[8];
 #pragma unroll
         for (int e = 0; e < 16; e += 2) {
-          const float p0 = ex2(fmaf(s[cc + e], p.scale_log2, neg_mu));
-          const float p1 = ex2(fmaf(s[cc + e + 1], p.scale_log2, neg_mu));
+          const float p0 = ex2(fmaf(s[cc + e], scale_log2, neg_mu));
+          const float p1 = ex2(fmaf(s[cc + e + 1], scale_log2, neg_mu));
           ls4[(e >> 1) & 3] += p0 + p1;
-          pk[e / 2] = pack_bf16x2(p0, p1);
+          pk[e / 2] = FP8 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
         }
         tmem_st8(s_addr + cc / 2, pk);      // P row over the consumed S columns
       }
@@ -384,21 +552,6 @@ __global__ void __launch_bounds__(224, kCtasPerSm)
           tmem_st32(lane_base + C::kOCol + cc, r);
         }
       }
-      // keys at or past this CTA's end may hold anything (past L: any bytes; past a
-      // row tile's last visible key in a paged cache: blocks never loaded, stale
-      // shared memory), even NaN: zero their V rows, which the PV MMA would
-      // otherwise multiply by p = 0
-      const int valid = tok_end - key0;
-      if (valid < kTok && warp == 0) {
-        const int ks = i % kStages;
-        if (!tc_wait(&bars[T_VFULL + ks], (i / kStages) & 1, abort_flag, p.status)) { ok = false; break; }
-        uint8_t* vst = smem + C::kVOff + ks * C::kTileBytes;
-        for (int idx = max(valid, 0) * 8 + lane; idx < kTok * 8; idx += 32)
-#pragma unroll
-          for (int hh = 0; hh < C::kHalves; ++hh)
-            *reinterpret_cast<uint4*>(vst + hh * C::kHalfBytes + idx * 16) = make_uint4(0, 0, 0, 0);
-        fence_proxy_async_smem();
-      }
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -410,7 +563,7 @@ __global__ void __launch_bounds__(224, kCtasPerSm)
     if (ok && tc_wait(&bars[T_OFINAL], 0, abort_flag, p.status) && !*abort_flag) {
       tc_fence_after();
       float* out = p.part_o + (row0 + row) * D;
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const float inv_l = l > 0.f ? v_mul / l : 0.f;
 #pragma unroll
       for (int cc = 0; cc < D; cc += 32) {
         uint32_t r[32];
@@ -445,9 +598,9 @@ __global__ void __launch_bounds__(224, kCtasPerSm)
   }
 }
 
-template <int D, bool PAGED>
+template <int D, bool PAGED, bool FP8>
 cudaError_t run_tc(const DecodeLaunch& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream) {
-  using C = TcCfg<D>;
+  using C = TcCfg<D, FP8>;
   const int G = a.Hq / a.Hkv;
   const int TT = decode_tc_tile_tokens(a.T, G);
   const int row_tiles = (a.T + TT - 1) / TT;
@@ -458,6 +611,8 @@ cudaError_t run_tc(const DecodeLaunch& a, const CUtensorMap& tk, const CUtensorM
   cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)TT, 1};
   if (encode_tmap_nd(&tq, a.q, 4, dims, str, box)) return cudaErrorInvalidValue;
   TcParams p;
+  p.k_scale = a.k_scale;
+  p.v_scale = a.v_scale;
   p.seqlens = a.seqlens;
   p.page_table = a.page_table;
   p.part_o = a.part_o;
@@ -477,7 +632,7 @@ cudaError_t run_tc(const DecodeLaunch& a, const CUtensorMap& tk, const CUtensorM
   p.max_seqlen = a.max_seqlen;
   p.scale_log2 = a.scale * kLog2e;
   p.causal = a.causal;
-  auto kern = decode_tc_kernel<D, PAGED>;
+  auto kern = decode_tc_kernel<D, PAGED, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   if ((long long)a.max_chunks * row_tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
@@ -491,8 +646,13 @@ cudaError_t run_tc(const DecodeLaunch& a, const CUtensorMap& tk, const CUtensorM
 cudaError_t launch_decode_tc(const DecodeLaunch& a, const CUtensorMap& tk, const CUtensorMap& tv,
                              cudaStream_t stream) {
   const bool paged = a.page_table != nullptr;
-  if (a.d == 128) return paged ? run_tc<128, true>(a, tk, tv, stream) : run_tc<128, false>(a, tk, tv, stream);
-  return paged ? run_tc<64, true>(a, tk, tv, stream) : run_tc<64, false>(a, tk, tv, stream);
+  if (a.fp8) {   // api.cu admits FP8 caches with d = 128 only
+    if (a.d != 128) return cudaErrorInvalidValue;
+    return paged ? run_tc<128, true, true>(a, tk, tv, stream) : run_tc<128, false, true>(a, tk, tv, stream);
+  }
+  if (a.d == 128)
+    return paged ? run_tc<128, true, false>(a, tk, tv, stream) : run_tc<128, false, false>(a, tk, tv, stream);
+  return paged ? run_tc<64, true, false>(a, tk, tv, stream) : run_tc<64, false, false>(a, tk, tv, stream);
 }
 
 }  // namespace kvattn

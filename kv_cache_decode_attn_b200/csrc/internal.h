@@ -17,10 +17,11 @@ constexpr int kDecodeTcTile = 64;  // tokens per K/V tile of the tensor-core dec
 // row groups each re-read the K/V fragments; up to 16 rows the warp-MMA kernel
 // streams at the HBM rate.
 constexpr int kDecodeMmaRows = 16;
-// FP8 caches have warp-MMA kernels only: at most this many rows per KV head.
+// FP8 caches run the warp-MMA kernels up to this many rows per KV head, and the
+// tensor-core kernel (converting each e4m3 tile to bf16 in shared memory) above.
 constexpr int kFp8MaxRows = 32;
 // Whether attn_decode runs the tensor-core split kernel for R rows per KV head.
-inline bool decode_uses_tc(int R, bool fp8) { return !fp8 && R > kDecodeMmaRows; }
+inline bool decode_uses_tc(int R, bool fp8) { return R > (fp8 ? kFp8MaxRows : kDecodeMmaRows); }
 
 // One CTA whose thread waits on an mbarrier nothing arrives at (bounded like every
 // wait of the library) and then sets DEV_TIMEOUT (csrc/selftest.cu).

@@ -542,6 +542,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool next_k = j + 1 < n_load;
         ok = wait_or_abort(&bars[B_VFULL + st], (gj / kVStages) & 1, abort_flag, p.status);
         if (!ok) break;
+        if constexpr (!kDenseKv<KV>) {
+          // V rows of keys >= L: any bytes (cache) or never loaded (paged); the PV MMAs
+          // would multiply them by p = 0.  Zeroed here, by the warp that consumes the V
+          // phases in order, before either PV of the tile is issued.
+          const int valid = __shfl_sync(0xffffffffu, itm.L, 0) - j * kBN;
+          if (valid < kBN) {
+            uint8_t* vst = smem + C::kVOff + st * C::kTileBytes;
+            for (int idx = max(valid, 0) * 8 + lane; idx < kBN * 8; idx += 32)
+#pragma unroll
+              for (int hh = 0; hh < C::kHalves; ++hh)
+                *reinterpret_cast<uint4*>(vst + hh * C::kHalfBytes + idx * 16) = make_uint4(0, 0, 0, 0);
+            fence_proxy_async_smem();
+            __syncwarp();
+          }
+        }
         if (j < n_kv0) {
           ok = pv_tile(0, st, j, it);
           if (!ok) break;
@@ -578,7 +593,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t s_addr = lane_base + C::s_col(t);
     const uint32_t o_addr = lane_base + C::o_col(t);
     int scnt = 0, it = 0;                               // S_FULL phases consumed, items done
-    int g_base = 0;                                     // K/V tiles of the previous items
     bool ok = true;
     for (;; ++it) {
     if (!wait_or_abort(&bars[B_QFULL], it & 1, abort_flag, p.status)) { ok = false; break; }
@@ -587,8 +601,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const Item itm = item_of<KV>(w, p, order);
     const int q_row = (2 * itm.qb + t) * kBM + row;
     const int nkv = t ? itm.n_load : itm.n_kv0;
-    const int g_item = g_base;
-    g_base += itm.n_load;
     float m = -INFINITY, l = 0.f;
     for (int j = 0; j < nkv; ++j) {
       if (!wait_or_abort(&bars[B_SFULL + t], (scnt++) & 1, abort_flag, p.status)) { ok = false; break; }
@@ -630,23 +642,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         m = m_new;
       }
       const float neg_mu = (m == -INFINITY) ? 0.f : -m;
-      if constexpr (!kDenseKv<KV>) {
-        // V rows of keys >= L: any bytes (cache) or never loaded (paged); the PV MMA
-        // would multiply them by p = 0.  The group whose PV reads the tile first zeroes
-        // them before it publishes any P: tile A for j < n_kv0 (PV_A(j) is issued before
-        // PV_B(j)), tile B for the tiles only it reads.
-        const int valid = itm.L - key0;
-        if (valid < kBN && (warp & 3) == 0 && (t == 0 || j >= itm.n_kv0)) {
-          const int gj = g_item + j, st = gj % kVStages;
-          if (!wait_or_abort(&bars[B_VFULL + st], (gj / kVStages) & 1, abort_flag, p.status)) { ok = false; break; }
-          uint8_t* vst = smem + C::kVOff + st * C::kTileBytes;
-          for (int idx = max(valid, 0) * 8 + lane; idx < kBN * 8; idx += 32)
-#pragma unroll
-            for (int hh = 0; hh < C::kHalves; ++hh)
-              *reinterpret_cast<uint4*>(vst + hh * C::kHalfBytes + idx * 16) = make_uint4(0, 0, 0, 0);
-          fence_proxy_async_smem();
-        }
-      }
       // O_t is stable here (PV_t(j-1) completed before S_t(j) did) and PV_t(j)
       // waits for this group's first arrival below
       // (16 columns at a time: the scores still occupy 128 registers)

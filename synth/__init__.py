@@ -97,6 +97,9 @@ WORKLOADS = {
     # eight new tokens per step (speculative verify): 64 query rows per KV head
     "decode_paged_t8": Decode("decode_paged_t8", B=8, T=8, Hq=64, Hkv=8, d=128, len_lo=32768,
                               len_hi=131072, paged=True),
+    # the same over an FP8 (e4m3) cache
+    "decode_paged_t8_fp8": Decode("decode_paged_t8_fp8", B=8, T=8, Hq=64, Hkv=8, d=128, len_lo=32768,
+                                  len_hi=131072, paged=True, fp8=True),
 }
 
 SEEDS = {name: 1000 + i for i, name in enumerate(WORKLOADS)}

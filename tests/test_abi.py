@@ -125,8 +125,7 @@ def test_decode_fp8_rejects_bad_arguments():
     assert call(vs=None) == kv.ATTN_ERR_INVALID_ARG
     assert call(q=None) == kv.ATTN_ERR_INVALID_ARG
     assert call(d=64) == kv.ATTN_ERR_UNSUPPORTED               # FP8 decode is built for d = 128
-    assert call(Hq=36, Hkv=1) == kv.ATTN_ERR_UNSUPPORTED       # 36 rows per KV head > 32
-    assert call(Hq=8, Hkv=1, T=5) == kv.ATTN_ERR_UNSUPPORTED   # 40 rows
+    assert call(Hq=256, Hkv=1) == kv.ATTN_ERR_UNSUPPORTED      # one token's heads exceed a 128-row tile
     assert call(wsb=16) == kv.ATTN_ERR_WORKSPACE
     assert call(T=4, msk=3) == kv.ATTN_ERR_INVALID_ARG
 

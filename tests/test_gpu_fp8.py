@@ -84,6 +84,48 @@ def test_fp8_decode_small_parity(paged, T, Hq, Hkv):
     check_lse(lse, lse_ref)
 
 
+@pytest.mark.parametrize("paged", [False, True])
+@pytest.mark.parametrize("T,Hq,Hkv", [(5, 8, 1), (8, 64, 8), (16, 64, 8), (33, 8, 2)])
+def test_fp8_decode_many_rows_tensor_core(paged, T, Hq, Hkv):
+    """More than 32 query rows per KV head (40, 64, 128, and 132 in two row tiles):
+    the tensor-core kernel, converting each e4m3 tile to bf16 in shared memory."""
+    d = 128
+    case = synth.decode_inputs(len(SMALL_LENS), T, Hq, Hkv, d, 0, 0, seed=900 + T * Hq, device="cuda", paged=paged,
+                               lengths=SMALL_LENS, spare_blocks=3, fp8=True)
+    host = host_copy(case)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = run_step(case, T, Hq, d, scale)
+    o_ref, lse_ref = oracle_step(host, T, scale)
+    check_o(o, o_ref)
+    check_lse(lse, lse_ref)
+
+
+@pytest.mark.parametrize("num_splits", [1, 3, 16])
+@pytest.mark.parametrize("causal", [True, False])
+def test_fp8_tensor_core_split_counts_bf16_out(num_splits, causal):
+    T, Hq, Hkv, d = 8, 32, 4, 128     # 64 rows per KV head
+    lens = [9, 700, 4100]
+    case = synth.decode_inputs(len(lens), T, Hq, Hkv, d, 0, 0, seed=78, device="cuda", lengths=lens, fp8=True)
+    host = host_copy(case)
+    o, lse = run_step(case, T, Hq, d, 0.09, causal=causal, num_splits=num_splits, o_dtype=torch.bfloat16)
+    o_ref, lse_ref = oracle_step(host, T, 0.09, causal)
+    check_o(o, o_ref)
+    check_lse(lse, lse_ref)
+
+
+def test_fp8_prompt_chunk_on_cached_prefix():
+    """A 200-token prompt chunk appended to FP8 cached prefixes (chunked prefill), paged."""
+    T, Hq, Hkv, d = 200, 8, 2, 128
+    lens = [0, 150, 1000, 3000]
+    case = synth.decode_inputs(len(lens), T, Hq, Hkv, d, 0, 0, seed=79, device="cuda", paged=True, lengths=lens,
+                               fp8=True)
+    host = host_copy(case)
+    o, lse = run_step(case, T, Hq, d, 0.088)
+    o_ref, lse_ref = oracle_step(host, T, 0.088)
+    check_o(o, o_ref)
+    check_lse(lse, lse_ref)
+
+
 @pytest.mark.parametrize("num_splits", [1, 3, 16])
 @pytest.mark.parametrize("causal", [True, False])
 @pytest.mark.parametrize("T,Hq,Hkv", [(4, 16, 4), (2, 8, 2)])     # 16 rows per KV head; 8 (transposed kernel)
@@ -259,7 +301,7 @@ def _sampled_rows_check(name, n_rows=12, seed=0):
     assert torch.isfinite(o).all() and torch.isfinite(lse).all()
 
 
-@pytest.mark.parametrize("name", ["decode_contig_fp8", "decode_paged_fp8"])
+@pytest.mark.parametrize("name", ["decode_contig_fp8", "decode_paged_fp8", "decode_paged_t8_fp8"])
 def test_fp8_full_size_workload_sampled_rows(name):
     _sampled_rows_check(name)
     torch.cuda.empty_cache()
