@@ -17,7 +17,8 @@
 //               policy (64-token tiles; contiguous: one 64-row box per 64
 //               columns of d; paged: one 16-row box per physical block, its
 //               page-table entry checked first).  K is released by S_j, V only by
-//               PV_j, so separate producers let the K ring run ahead;
+//               PV_j, so separate producers let the K ring run ahead (FP8:
+//               warps 7 and 6 copy and convert, see below);
 //   warp 5      MMA issuer: S_j = Q K_j^T (SS) into one of two TMEM S buffers,
 //               O += P_j V_j (P read from TMEM, where the softmax wrote it over
 //               the consumed S columns).  S_{j+1} is issued before PV_j, so the
@@ -49,6 +50,11 @@ constexpr float kLn2 = 0.6931471805599453f;
 
 constexpr int kStages = 2;    // K/V ring stages (S is double-buffered in TMEM)
 constexpr int kCtasPerSm = 2;   // shared memory and TMEM of one CTA
+// FP8 adds warp 7: the K converter runs on warp 7 and the V converter on warp 6, so
+// that neither shares an SM sub-partition (warp index mod 4) with softmax warps 0
+// and 1, the only ones a tile of up to 64 rows uses.
+template <bool FP8>
+constexpr int tc_threads() { return FP8 ? 256 : 224; }
 
 // FP8: the cache holds e4m3 codes.  The copies land in a ring of raw stages; the K
 // (V) producer warp then converts each raw tile into one f16 K (V) tile in the
@@ -155,7 +161,7 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t x) {
 }
 
 template <int D, bool PAGED, bool FP8>
-__global__ void __launch_bounds__(224, kCtasPerSm)
+__global__ void __launch_bounds__(tc_threads<FP8>(), kCtasPerSm)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const TcParams p) {
   using C = TcCfg<D, FP8>;
@@ -247,12 +253,13 @@ __global__ void __launch_bounds__(224, kCtasPerSm)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (FP8 && (warp == 4 || warp == 6)) {
+  if (FP8 && (warp == 7 || warp == 6)) {
     // ------------------------------------------------ FP8 producers and converters
     // Lane 0 copies raw e4m3 tiles into a 2-stage ring; the whole warp converts each
-    // raw tile into the one bf16 operand tile once the MMA has finished reading the
-    // previous one, then refills the raw stage it has just read.
-    const bool is_k = warp == 4;
+    // raw tile into the one f16 operand tile once the MMA has finished reading the
+    // previous one, then refills the raw stage it has just read.  Warp 7 handles K
+    // (and Q), warp 6 V; warp 4 has no work.
+    const bool is_k = warp == 7;
     const CUtensorMap* map = is_k ? &tmK : &tmV;
     uint8_t* raw_ring = smem + (is_k ? C::kRawKOff : C::kRawVOff);
     uint8_t* conv = smem + (is_k ? C::kKOff : C::kVOff);
@@ -334,7 +341,7 @@ __global__ void __launch_bounds__(224, kCtasPerSm)
       if (is_k) mbar_wait(&bars[T_Q], 0);
       for (int i = max(0, issued - kStages); i < issued; ++i) mbar_wait(&bars[full0 + i % kStages], (i / kStages) & 1);
     }
-  } else if (warp == 4 || warp == 6) {
+  } else if (!FP8 && (warp == 4 || warp == 6)) {
     // ------------------------------------------------------------- TMA producers
     if (lane == 0) {
       const bool is_k = warp == 4;
@@ -637,7 +644,7 @@ cudaError_t run_tc(const DecodeLaunch& a, const CUtensorMap& tk, const CUtensorM
   if (e != cudaSuccess) return e;
   if ((long long)a.max_chunks * row_tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
   dim3 grid(a.max_chunks * row_tiles, a.Hkv, a.B);
-  kern<<<grid, 224, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  kern<<<grid, tc_threads<FP8>(), C::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
