@@ -8,16 +8,16 @@
 // loaded for the item.  Warp roles (12 warps, three warpgroups):
 //   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread i of a
 //              group owns query row i, which is TMEM lane i of its S and O;
-//   warp 8     TMA producer: Q_A and Q_B per item (the next item's Q is
-//              prefetched into L2 early), K_j and V_j through a ring (2
-//              stages at d = 128, 4 at d = 64) that runs on across items; K
-//              and V of a stage are released separately (K after the second S
-//              MMA, V after the second PV);
+//   warps 8,10 TMA producers: warp 8 loads Q_A and Q_B per item (the next
+//              item's Q is prefetched into L2 early) and the K tiles, warp 10
+//              the V tiles, each through its own ring (2 stages at d = 128, 4
+//              at d = 64) that runs on across items; K is released after the
+//              second S MMA reading it, V after the second PV;
 //   warp 9     MMA issuer: the whole warp runs the loop, one elected lane
 //              issues (operands stay warp-uniform, so each MMA costs the
 //              issuing warp only a few instructions on a sub-partition it
 //              shares with two busy softmax warps);
-//   warps 10-11 complete the producer warpgroup for the register split.
+//   warp 11    completes the producer warpgroup for the register split.
 // TMEM (512 columns): S_A | S_B | O_A | O_B.  Each softmax group reads its S row,
 // turns it into bf16 probabilities P and writes P back over the first half of
 // the same S columns, in two halves of 64 keys: the PV MMA of the first half
@@ -77,12 +77,6 @@ namespace {
 constexpr int kBM = 128;          // query rows per tile (two tiles per CTA)
 constexpr int kBN = 128;          // keys per K/V tile
 constexpr int kThreads = 384;     // 8 softmax warps + TMA warp + MMA warp + 2 idle warps (a full warpgroup)
-// Register split (setmaxnreg): 384 threads launch with 168 registers each; the producer
-// warpgroup (TMA, MMA, two idle warps) gives back down to kRegsIo so each softmax thread
-// can hold its 128 scores and the exponential temporaries without spilling.
-constexpr int kRegsIo = 72;
-constexpr int kRegsSoftmax = 216;
-static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsIo <= 168 * kThreads, "register split exceeds the launch");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 of the largest allowed p
@@ -119,8 +113,8 @@ struct PrefillCfg {
 
 enum Bar {
   B_QFULL = 0,
-  B_QEMPTY = 1,                     // all MMAs of an item done and every softmax warp has read
-                                    // the item (9 arrivals): its Q tiles may be replaced
+  B_QEMPTY = 1,                     // all MMAs of an item done and every softmax warp and the V
+                                    // producer have read the item (10 arrivals): its Q may be replaced
   B_KFULL = 2,                      // +K stage
   B_KEMPTY = B_KFULL + kMaxStages,  // +K stage: both S MMAs reading this K stage are done
   B_VFULL = B_KEMPTY + kMaxStages,  // +V stage
@@ -138,6 +132,21 @@ static_assert(B_COUNT * 8 + 8 + 4 * kItemSlots <= 256, "barrier block");
 // Where K and V come from.
 // KV_DENSE_GROUPED: the dense form with its items in the cached forms' order.
 enum KvSource { KV_DENSE = 0, KV_CACHE = 1, KV_PAGED = 2, KV_DENSE_GROUPED = 3 };
+
+// Register split (setmaxnreg): 384 threads launch with 168 registers each; the producer
+// warpgroup (two TMA warps, the MMA warp and one more) gives back down to regs_io() so
+// each softmax thread can hold its 128 scores and the exponential temporaries.  Chosen
+// per form by ptxas's spill report: the dense d = 128 softmax needs 216 registers, the
+// other forms spill less with 208 and 88 for the producers (the cached forms' producers
+// also track the sequence lengths and page-table entries).
+template <int D, int KV>
+constexpr int regs_softmax() { return D == 128 && KV == KV_DENSE ? 216 : 208; }
+template <int D, int KV>
+constexpr int regs_io() { return D == 128 && KV == KV_DENSE ? 72 : 88; }
+static_assert(2 * 128 * regs_softmax<128, KV_DENSE>() + 128 * regs_io<128, KV_DENSE>() <= 168 * kThreads,
+              "register split exceeds the launch");
+static_assert(2 * 128 * regs_softmax<64, KV_PAGED>() + 128 * regs_io<64, KV_PAGED>() <= 168 * kThreads,
+              "register split exceeds the launch");
 template <int KV>
 constexpr bool kDenseKv = KV == KV_DENSE || KV == KV_DENSE_GROUPED;
 
@@ -292,7 +301,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // work item of the CTA's it-th item in slot it % kItemSlots, published by the producer
   // before that item's Q copies complete B_QFULL phase it; -1 = no more work.  The slot
   // is written again for item it + kItemSlots only after B_QEMPTY of item
-  // it + kItemSlots - 1, which every softmax warp reaches after reading item it.
+  // it + kItemSlots - 1, which every softmax warp and the V producer reach after
+  // reading item it.
   volatile int* item_slot = reinterpret_cast<volatile int*>(tmem_slot + 2);
   int* order_smem = reinterpret_cast<int*>(smem + C::kOrderOff);
   const int* order = (!kDenseKv<KV> && p.B <= C::kMaxOrdered) ? order_smem : nullptr;
@@ -313,9 +323,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[B_QFULL], 1);
-    // the MMA warp's commit and one arrival per softmax warp: B_QFULL then never runs
-    // two phases ahead of a softmax warp (a parity wait would miss the phase it wants)
-    mbar_init(&bars[B_QEMPTY], 1 + 8);
+    // the MMA warp's commit and one arrival per softmax warp and from the V producer:
+    // B_QFULL then never runs two phases ahead of a warp that reads the item (a parity
+    // wait would miss the phase it wants)
+    mbar_init(&bars[B_QEMPTY], 1 + 8 + 1);
     for (int s = 0; s < C::kKStages; ++s) {
       mbar_init(&bars[B_KFULL + s], 1);
       mbar_init(&bars[B_KEMPTY + s], 1);
@@ -344,139 +355,132 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   if (warp >= 8) {
-  reg_dealloc<kRegsIo>();
-  if (warp == 8) {
-    // ------------------------------------------------------------- TMA producer
+  reg_dealloc<regs_io<D, KV>()>();
+  if (warp == 8 || warp == 10) {
+    // ------------------------------------------------------------- TMA producers
+    // Warp 8 loads Q per item and the K ring, warp 10 the V ring.  Each ring runs on
+    // across items, so a K copy never waits for a V stage that the PV MMAs still read.
+    // Paged caches: lane jb < 8 of the warp reads page-table entry jb of a tile (one tile
+    // ahead) and copies that physical block, so the eight blocks of a tile are handled in
+    // parallel instead of one after another by a single thread.
+    const bool is_k = warp == 8;
+    const CUtensorMap* map = is_k ? &tmK : &tmV;
+    const int stages = is_k ? C::kKStages : C::kVStages;
+    const int full0 = is_k ? B_KFULL : B_VFULL, empty0 = is_k ? B_KEMPTY : B_VEMPTY;
+    uint8_t* const ring = smem + (is_k ? C::kKOff : C::kVOff);
     if (lane == 0) {
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
-      const uint64_t keep = policy_evict_last();    // K/V tiles are re-read by other query blocks and heads
-      const uint64_t once = policy_evict_first();
-      constexpr int kKStages = C::kKStages, kVStages = C::kVStages;
-      int g = 0, it = 0, q_loaded = 0;              // K/V tiles loaded, items started, Q loads issued
-      int last_k[kKStages], last_v[kVStages];   // last K / V tile whose copy was issued per stage
+      prefetch_tmap(map);
+      if (is_k) prefetch_tmap(&tmQ);
+    }
+    const uint64_t keep = policy_evict_last();    // K/V tiles are re-read by other query blocks and heads
+    const uint64_t once = policy_evict_first();
+    constexpr int kBlocks = kBN / kPageTokens;
+    int g = 0, it = 0, q_loaded = 0;              // tiles loaded, items started, Q loads issued
+    int last[kMaxStages];                         // last tile whose copy was issued per stage
 #pragma unroll
-      for (int i = 0; i < kKStages; ++i) last_k[i] = -1;
-#pragma unroll
-      for (int i = 0; i < kVStages; ++i) last_v[i] = -1;
-      bool ok = true, clean_end = false;
-      for (int w = blockIdx.x;; ++it) {
+    for (int i = 0; i < kMaxStages; ++i) last[i] = -1;
+    bool ok = true, clean_end = false;
+    for (int w = blockIdx.x;; ++it) {
+      Item itm;
+      int w_next = 0;
+      if (is_k) {
         // Q of the previous item no longer read (this also means its copy landed), and
-        // that item read by every softmax warp
+        // that item read by every softmax warp and by the V producer
         if (it > 0 && !wait_or_abort(&bars[B_QEMPTY], (it - 1) & 1, abort_flag, p.status)) break;
         if (w >= p.n_items) {
           // no more work: complete B_QFULL phase `it` without a copy
-          item_slot[it % kItemSlots] = -1;
-          mbar_arrive(&bars[B_QFULL]);
+          if (lane == 0) {
+            item_slot[it % kItemSlots] = -1;
+            mbar_arrive(&bars[B_QFULL]);
+          }
           clean_end = true;
           break;
         }
-        item_slot[it % kItemSlots] = w;
-        const Item itm = item_of<KV>(w, p, order);
-        const int kvh = itm.h / p.G;
-        const int w_next = (int)gridDim.x + (int)atomicAdd(p.next_item, 1u);
-        mbar_arrive_expect_tx(&bars[B_QFULL], 2 * C::kTileBytes);
+        if (lane == 0) item_slot[it % kItemSlots] = w;
+        itm = item_of<KV>(w, p, order);
+        if (lane == 0) w_next = (int)gridDim.x + (int)atomicAdd(p.next_item, 1u);
+        w_next = __shfl_sync(0xffffffffu, w_next, 0);
         ++q_loaded;
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
-#pragma unroll
-          for (int hh = 0; hh < C::kHalves; ++hh)
-            tma_load_4d(smem + C::kQOff + t * C::kTileBytes + hh * C::kHalfBytes, &tmQ, &bars[B_QFULL], hh * 64,
-                        itm.h, (2 * itm.qb + t) * kBM, itm.b, once);
-        if (w_next < p.n_items) {                   // warm L2 with the next item's Q
-          const Item nx = item_of<KV>(w_next, p, order);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&bars[B_QFULL], 2 * C::kTileBytes);
 #pragma unroll
           for (int t = 0; t < 2; ++t)
 #pragma unroll
-            for (int hh = 0; hh < C::kHalves; ++hh) tma_prefetch_4d(&tmQ, hh * 64, nx.h, (2 * nx.qb + t) * kBM, nx.b);
-        }
-        // paged: the physical blocks of tile t, read one tile ahead (the page-table
-        // latency then overlaps the wait for a free stage instead of delaying the copy)
-        constexpr int kBlocks = kBN / kPageTokens;
-        int ids[kBlocks];
-        int nb = 0;
-        auto read_ids = [&](int t) {
-          nb = min(kBlocks, (itm.L - t * kBN + kPageTokens - 1) / kPageTokens);
-          const int32_t* tab = p.page_table + (size_t)itm.b * p.max_blocks + t * kBlocks;
-#pragma unroll
-          for (int jb = 0; jb < kBlocks; ++jb) ids[jb] = jb < nb ? __ldg(tab + jb) : 0;
-        };
-        if constexpr (KV == KV_PAGED) read_ids(0);
-        for (int t = 0; t < itm.n_load; ++t, ++g) {
-          const int ks = g % kKStages, vs = g % kVStages;
-          // K of a stage is released after the second S MMA reading it, V after the
-          // second PV MMA, so the next K tiles land while the current PVs still run
-          if (g >= kKStages &&
-              !wait_or_abort(&bars[B_KEMPTY + ks], ((g / kKStages) - 1) & 1, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          last_k[ks] = g;
-          if constexpr (KV != KV_PAGED) {
-            mbar_arrive_expect_tx(&bars[B_KFULL + ks], C::kTileBytes);
-#pragma unroll
             for (int hh = 0; hh < C::kHalves; ++hh)
-              tma_load_4d(smem + C::kKOff + ks * C::kTileBytes + hh * C::kHalfBytes, &tmK, &bars[B_KFULL + ks],
-                          hh * 64, kvh, t * kBN, itm.b, keep);
-            if (g >= kVStages &&
-                !wait_or_abort(&bars[B_VEMPTY + vs], ((g / kVStages) - 1) & 1, abort_flag, p.status)) {
-              ok = false;
-              break;
-            }
-            last_v[vs] = g;
-            mbar_arrive_expect_tx(&bars[B_VFULL + vs], C::kTileBytes);
+              tma_load_4d(smem + C::kQOff + t * C::kTileBytes + hh * C::kHalfBytes, &tmQ, &bars[B_QFULL], hh * 64,
+                          itm.h, (2 * itm.qb + t) * kBM, itm.b, once);
+          if (w_next < p.n_items) {                 // warm L2 with the next item's Q
+            const Item nx = item_of<KV>(w_next, p, order);
 #pragma unroll
-            for (int hh = 0; hh < C::kHalves; ++hh)
-              tma_load_4d(smem + C::kVOff + vs * C::kTileBytes + hh * C::kHalfBytes, &tmV, &bars[B_VFULL + vs],
-                          hh * 64, kvh, t * kBN, itm.b, keep);
-          } else {
-            // one 16-row box per physical block holding keys of this tile below L
-#pragma unroll
-            for (int jb = 0; jb < kBlocks; ++jb) {
-              if (jb < nb && (ids[jb] < 0 || ids[jb] >= p.num_blocks)) {
-                atomicOr(p.status, DEV_PAGE_ID);
-                ids[jb] = 0;   // keep the byte count; the result is flagged invalid
-              }
-            }
-            const uint32_t bytes = nb * C::kHalves * kPageTokens * 128;
-            mbar_arrive_expect_tx(&bars[B_KFULL + ks], bytes);
-#pragma unroll
-            for (int jb = 0; jb < kBlocks; ++jb) {
-              if (jb >= nb) break;
+            for (int t = 0; t < 2; ++t)
 #pragma unroll
               for (int hh = 0; hh < C::kHalves; ++hh)
-                tma_load_3d(smem + C::kKOff + ks * C::kTileBytes + hh * C::kHalfBytes + jb * kPageTokens * 128, &tmK,
-                            &bars[B_KFULL + ks], hh * 64, kvh, ids[jb] * kPageTokens, keep);
-            }
-            if (g >= kVStages &&
-                !wait_or_abort(&bars[B_VEMPTY + vs], ((g / kVStages) - 1) & 1, abort_flag, p.status)) {
-              ok = false;
-              break;
-            }
-            last_v[vs] = g;
-            mbar_arrive_expect_tx(&bars[B_VFULL + vs], bytes);
-#pragma unroll
-            for (int jb = 0; jb < kBlocks; ++jb) {
-              if (jb >= nb) break;
-#pragma unroll
-              for (int hh = 0; hh < C::kHalves; ++hh)
-                tma_load_3d(smem + C::kVOff + vs * C::kTileBytes + hh * C::kHalfBytes + jb * kPageTokens * 128, &tmV,
-                            &bars[B_VFULL + vs], hh * 64, kvh, ids[jb] * kPageTokens, keep);
-            }
-            if (t + 1 < itm.n_load) read_ids(t + 1);
+                tma_prefetch_4d(&tmQ, hh * 64, nx.h, (2 * nx.qb + t) * kBM, nx.b);
           }
         }
-        if (!ok) break;
-        w = w_next;
+      } else {
+        // the item the K producer published (the V copies of an item follow its Q copies)
+        if (!wait_or_abort(&bars[B_QFULL], it & 1, abort_flag, p.status)) break;
+        const int wi = item_slot[it % kItemSlots];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[B_QEMPTY]);
+        if (wi < 0) {
+          clean_end = true;
+          break;
+        }
+        itm = item_of<KV>(wi, p, order);
       }
-      // no copy may still be landing in shared memory when the CTA exits (after a clean
-      // end, the wait on B_QEMPTY above already covered the last Q copy)
-      if (!clean_end && q_loaded > 0) mbar_wait(&bars[B_QFULL], (q_loaded - 1) & 1);
-      for (int i = 0; i < kKStages; ++i)
-        if (last_k[i] >= 0) mbar_wait(&bars[B_KFULL + i], (last_k[i] / kKStages) & 1);
-      for (int i = 0; i < kVStages; ++i)
-        if (last_v[i] >= 0) mbar_wait(&bars[B_VFULL + i], (last_v[i] / kVStages) & 1);
+      const int kvh = itm.h / p.G;
+      // paged: this lane's physical block of tile t (lanes >= 8 and blocks past L: none)
+      auto read_id = [&](int t) -> int {
+        const int nb = min(kBlocks, (itm.L - t * kBN + kPageTokens - 1) / kPageTokens);
+        return lane < nb ? __ldg(p.page_table + (size_t)itm.b * p.max_blocks + t * kBlocks + lane) : -1;
+      };
+      int id = 0;
+      if constexpr (KV == KV_PAGED) id = read_id(0);
+      for (int t = 0; t < itm.n_load; ++t, ++g) {
+        const int s = g % stages;
+        if (g >= stages && !wait_or_abort(&bars[empty0 + s], ((g / stages) - 1) & 1, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        last[s] = g;
+        uint8_t* const dst = ring + s * C::kTileBytes;
+        if constexpr (KV != KV_PAGED) {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&bars[full0 + s], C::kTileBytes);
+#pragma unroll
+            for (int hh = 0; hh < C::kHalves; ++hh)
+              tma_load_4d(dst + hh * C::kHalfBytes, map, &bars[full0 + s], hh * 64, kvh, t * kBN, itm.b, keep);
+          }
+        } else {
+          // one 16-row box per 64 columns of d and physical block holding keys of this tile below L
+          const int nb = min(kBlocks, (itm.L - t * kBN + kPageTokens - 1) / kPageTokens);
+          int blk = id;
+          if (lane < nb && (blk < 0 || blk >= p.num_blocks)) {
+            atomicOr(p.status, DEV_PAGE_ID);
+            blk = 0;   // keep the byte count; the result is flagged invalid
+          }
+          if (lane == 0) mbar_arrive_expect_tx(&bars[full0 + s], nb * C::kHalves * kPageTokens * 128);
+          __syncwarp();
+          if (lane < nb) {
+#pragma unroll
+            for (int hh = 0; hh < C::kHalves; ++hh)
+              tma_load_3d(dst + hh * C::kHalfBytes + lane * kPageTokens * 128, map, &bars[full0 + s], hh * 64, kvh,
+                          blk * kPageTokens, keep);
+          }
+          if (t + 1 < itm.n_load) id = read_id(t + 1);
+        }
+      }
+      if (!ok) break;
+      w = w_next;
+    }
+    // no copy may still be landing in shared memory when the CTA exits (after a clean
+    // end, the wait on B_QEMPTY above already covered the last Q copy)
+    if (lane == 0) {
+      if (is_k && !clean_end && q_loaded > 0) mbar_wait(&bars[B_QFULL], (q_loaded - 1) & 1);
+      for (int i = 0; i < stages; ++i)
+        if (last[i] >= 0) mbar_wait(&bars[full0 + i], (last[i] / stages) & 1);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------- MMA issuer
@@ -599,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   } else {
-    reg_alloc<kRegsSoftmax>();
+    reg_alloc<regs_softmax<D, KV>()>();
     // -------------------------------------------------- softmax warps 0-7
     const int t = warp >> 2;                            // query tile of this group
     const int row = (warp & 3) * 32 + lane;             // TMEM lane == query row in the tile
@@ -840,7 +844,8 @@ cudaError_t run_prefill(const PrefillLaunch& a, cudaStream_t stream) {
   // whose launch register count could not cover the split
   cudaFuncAttributes fa;
   if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
-  if (fa.numRegs * kThreads < 2 * 128 * kRegsSoftmax + 128 * kRegsIo) return cudaErrorInvalidConfiguration;
+  if (fa.numRegs * kThreads < 2 * 128 * regs_softmax<D, KV>() + 128 * regs_io<D, KV>())
+    return cudaErrorInvalidConfiguration;
   // persistent: one CTA per SM (each owns all 512 TMEM columns)
   int dev = 0, sms = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
