@@ -239,7 +239,7 @@ def decode_kernel(wd):
     """(name, source files) of the kernel attn_decode picks for this shape: bf16 up
     to 16 query rows per KV head on warp-level MMAs, more on tcgen05; FP8 up to
     8 rows on the transposed-product kernel, up to 32 on the split kernel, more on
-    tcgen05 (e4m3 tiles converted to bf16 in shared memory)."""
+    tcgen05 (e4m3 tiles converted to f16 in shared memory)."""
     R = wd.Hq // wd.Hkv * wd.T
     if wd.fp8:
         if R <= 8:
@@ -370,12 +370,12 @@ def run_ours(args, world, rank, local):
     peaks, peak_src = load_peaks()
     pf_kernel_tflops = flops / (pf_ms / K * 1e-3) / 1e12          # per launch, this rank
     dec_kernel_gbs = dbytes / (dec_ms / K * 1e-3) / 1e9
-    traffic = load_traffic(args.workload, wd)
+    traffic = load_traffic(args.workload, wd, wp)
     roof_pf = {"bound": "tensor", "achieved": round(pf_kernel_tflops, 1), "peak": peaks["bf16_tflops"],
                "unit": "TFLOP/s", "frac": round(pf_kernel_tflops / peaks["bf16_tflops"], 4),
                "frac_of_sustained": round(pf_kernel_tflops / peaks["bf16_tflops_sustained"], 4),
                "peak_source": f"{peak_src} (bf16 burst)", "traffic": traffic.get("prefill"),
-               "kernel": "prefill_kernel<128>", "flops_per_launch": flops,
+               "kernel": f"prefill_kernel<{wp.d}>", "flops_per_launch": flops,
                "launch_ms": round(pf_ms / K, 4)}
     # the decode call is HBM-bound unless its flops per byte pass the ridge (many new tokens: chunked prefill)
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
@@ -600,7 +600,7 @@ def source_hash(files) -> str:
     return h.hexdigest()[:16]
 
 
-def load_traffic(workload, wd):
+def load_traffic(workload, wd, wp):
     """Per-launch DRAM bytes (ncu dram__bytes_read.sum + dram__bytes_write.sum,
     summed over the leg's kernels) from the committed profile summary, for this
     workload only, and kept only while the kernel sources it was measured on are
@@ -612,7 +612,7 @@ def load_traffic(workload, wd):
     except (OSError, ValueError, KeyError):
         return {}
     prefill_cache = workload in PREFILL_CACHE_SETS
-    want = {"prefill": ("prefill_kernel<128>", ("prefill.cu",)),
+    want = {"prefill": (f"prefill_kernel<{wp.d}>", ("prefill.cu",)),
             "decode": (decode_kernel_name(wd, True), ("prefill.cu",)) if prefill_cache else decode_kernel(wd)}
     out = {}
     for e in entries:

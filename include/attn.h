@@ -216,11 +216,15 @@ ATTN_API int kv_append(void* k_cache, void* v_cache, const void* k_new, const vo
  *                     rows are NaN and ATTN_DEV_SCALE is set
  *   everything else   as for attn_decode, including the workspace size
  *                     (attn_decode_workspace_bytes with the same arguments)
- * Built for d = 128 and at most 32 query rows per KV head ((Hq / Hkv) * T);
- * other shapes return ATTN_ERR_UNSUPPORTED.  The products run on f16 tensor
- * cores: every e4m3 value is exact in f16, q is rounded to f16 (exact for bf16
- * values of magnitude 2^-14 .. 65504; larger magnitudes overflow) and the
- * softmax weights are rounded to f16 before the P V product.
+ * Built for d = 128 (other d return ATTN_ERR_UNSUPPORTED) and, like
+ * attn_decode, for Hq / Hkv <= 128 and any T.  Up to 32 query rows per KV head
+ * ((Hq / Hkv) * T) run on warp-level f16 MMAs that convert the codes in
+ * registers; more rows run on the tcgen05 tensor cores in row tiles of at most
+ * 128 rows, the e4m3 tiles converted to f16 in shared memory.  Either way the
+ * products are f16 x f16 with fp32 accumulation: every e4m3 value is exact in
+ * f16, q is rounded to f16 (exact for bf16 values of magnitude 2^-14 .. 65504;
+ * larger magnitudes overflow) and the softmax weights are rounded to f16 before
+ * the P V product.
  */
 ATTN_API int attn_decode_fp8(const void* q, const void* k_cache, const void* v_cache, const float* k_scale,
                              const float* v_scale, const int32_t* seqlens_k, const int32_t* page_table,
