@@ -157,7 +157,10 @@ ATTN_API size_t attn_decode_workspace_bytes(int B, int T, int Hq, int Hkv, int d
  *                   grid and the workspace); 0 = the cache capacity
  *   o           device [B, T, Hq, d] of o_dtype;  lse  device fp32 [B, Hq, T] or NULL
  *   scale, causal   as for attn_prefill; causal with T == 1 equals non-causal
- *   num_splits  0 = automatic chunking; n > 0 = split every sequence's keys
+ *   num_splits  0 = automatic chunking (on the tensor-core kernel with one row
+ *               tile per KV head and B <= 128: chunks apportioned over the
+ *               sequences by their lengths on the device, so the work items fill
+ *               the GPU's CTA slots evenly); n > 0 = split every sequence's keys
  *               into at most n chunks
  *   workspace   device memory of at least attn_decode_workspace_bytes(...) bytes,
  *               16-byte aligned; contents on entry do not matter

@@ -81,7 +81,8 @@ namespace {
 
 struct DecodeLayout {
   int R, chunk, max_chunks;
-  size_t o_bytes, lse_offset, total;
+  int balanced, n_chunks;   // balanced split: chunks over the batch (per KV head)
+  size_t o_bytes, lse_offset, plan_offset, total;
 };
 
 bool decode_layout(int B, int T, int Hq, int Hkv, int d, int max_seqlen_k, int num_splits, bool fp8,
@@ -92,10 +93,19 @@ bool decode_layout(int B, int T, int Hq, int Hkv, int d, int max_seqlen_k, int n
   L.R = (Hq / Hkv) * T;
   L.chunk = decode_chunk_tokens(B, T, Hq / Hkv, Hkv, max_seqlen_k, num_splits, fp8);
   L.max_chunks = (max_seqlen_k + L.chunk - 1) / L.chunk;
-  const size_t items = (size_t)B * Hkv * L.max_chunks;
+  L.balanced = decode_balanced(B, T, Hq / Hkv, num_splits, fp8) ? 1 : 0;
+  L.n_chunks = 0;
+  size_t items = (size_t)B * Hkv * L.max_chunks;
+  if (L.balanced) {
+    // every sequence gets at least one chunk of the batch's n_chunks
+    L.n_chunks = decode_balanced_chunks(B, Hkv);
+    L.max_chunks = L.n_chunks - B + 1;   // most chunks one (sequence, KV head) can get
+    items = (size_t)L.n_chunks * Hkv;
+  }
   L.o_bytes = items * L.R * d * sizeof(float);
   L.lse_offset = (L.o_bytes + 255) & ~size_t(255);
-  L.total = L.lse_offset + items * L.R * sizeof(float);
+  L.plan_offset = (L.lse_offset + items * L.R * sizeof(float) + 255) & ~size_t(255);
+  L.total = L.plan_offset + (L.balanced ? (size_t)B * 3 * sizeof(int) : 0);
   *out = L;
   return true;
 }
@@ -252,6 +262,9 @@ int decode_impl(const void* q, const void* k_cache, const void* v_cache, const f
   a.max_chunks = L.max_chunks;
   a.part_o = static_cast<float*>(workspace);
   a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + L.lse_offset);
+  a.balanced = L.balanced;
+  a.n_chunks = L.n_chunks;
+  a.plan = L.balanced ? reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + L.plan_offset) : nullptr;
   a.status = st;
   a.fp8 = fp8 ? 1 : 0;
   a.k_scale = k_scale;

@@ -485,20 +485,26 @@ __global__ void __launch_bounds__(256, kBatch >= 8 ? 2 : 5) decode_combine_kerne
   const int b = row / (p.Hq * p.T);
   const int g = h / p.G, r = t * p.G + (h - g * p.G);
   bool bad = true;
-  int nc = 0;
+  int nc = 0, L = 0;
   if (live) {
-    const int L = seqlens[b];
+    L = seqlens[b];
     bad = seqlen_bad(L, p.T, p.max_seqlen, paged != 0, p.capacity, p.max_blocks);
-    if (!bad) nc = (L + p.chunk - 1) / p.chunk;
+    if (!bad && !p.balanced) nc = (L + p.chunk - 1) / p.chunk;
   }
   grid_dependency_wait();   // launched early (programmatic dependent launch): the partials are ready after this
+  // chunks of this (b, g): fixed length, or the balanced plan the split kernel wrote
+  size_t item0 = ((size_t)b * p.Hkv + g) * p.max_chunks;
+  if (p.balanced && live && !bad) {
+    const int first = p.plan[3 * b], n_b = p.plan[3 * b + 1], chunk_b = p.plan[3 * b + 2];
+    nc = (L + chunk_b - 1) / chunk_b;
+    item0 = (size_t)p.Hkv * first + (size_t)g * n_b;
+  }
 
   float acc[kPer];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
   float lse_row = -INFINITY;
   if (nc > 0) {
-    const size_t item0 = ((size_t)b * p.Hkv + g) * p.max_chunks;
     const float* lse0 = part_lse + item0 * p.R + r;            // chunk c at lse0[c * R]
     const float* src0 = part_o + (item0 * p.R + r) * D + lane * kPer;
     const size_t cstride = (size_t)p.R * D;                    // floats between consecutive chunks of this row
@@ -642,6 +648,17 @@ int decode_chunk_tokens(int B, int T, int G, int Hkv, int max_seqlen, int num_sp
   return chunk < kDecodeTcTile ? kDecodeTcTile : chunk;
 }
 
+int decode_balanced_chunks(int B, int Hkv) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+    cudaGetLastError();   // no device here (workspace sizing on a host without one): a B200's 148 SMs
+    sms = 148;
+  }
+  const int n = kBalancedItemsPerSlot * kDecodeTcCtasPerSm * sms / Hkv;
+  return n > B ? n : B;
+}
+
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
   const bool paged = a.page_table != nullptr;
   const int G = a.Hq / a.Hkv, R = G * a.T;
@@ -667,6 +684,8 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
   sp.max_seqlen = a.max_seqlen;
   sp.scale_log2 = a.scale * kLog2e;
   sp.causal = a.causal;
+  sp.balanced = a.balanced;
+  sp.plan = a.plan;
 
   // K/V viewed as 3-D {d, Hkv, rows}: rows = B * capacity (contiguous) or num_blocks * 16 (paged)
   const uint64_t rows = paged ? (uint64_t)a.num_blocks * kPageTokens : (uint64_t)a.B * a.capacity;

@@ -49,7 +49,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 constexpr int kStages = 2;    // K/V ring stages (S is double-buffered in TMEM)
-constexpr int kCtasPerSm = 2;   // shared memory and TMEM of one CTA
+constexpr int kCtasPerSm = kDecodeTcCtasPerSm;   // shared memory and TMEM of one CTA
 // FP8 adds warp 7: the K converter runs on warp 7 and the V converter on warp 6, so
 // that neither shares an SM sub-partition (warp index mod 4) with softmax warps 0
 // and 1, the only ones a tile of up to 64 rows uses.
@@ -76,7 +76,9 @@ struct TcCfg {
   static constexpr int kRawKOff = kVOff + kOperandStages * kTileBytes;   // FP8: raw K stages
   static constexpr int kRawVOff = kRawKOff + (FP8 ? kStages * kRawBytes : 0);
   static constexpr int kBarOff = kRawVOff + (FP8 ? kStages * kRawBytes : 0);
-  static constexpr int kSmemBytes = kBarOff + 256 + 1024;
+  static constexpr int kPlanOff = kBarOff + 256;             // balanced split: the plan, built per CTA
+  static constexpr int kPlanBytes = kBalancedMaxB * 4 * 4;   // length, base share, chunks, first chunk
+  static constexpr int kSmemBytes = kPlanOff + kPlanBytes + 1024;
   static constexpr int kSCols = kTok;                        // one S buffer (fp32 scores of a tile)
   static constexpr int kOCol = 2 * kSCols;                   // S0 | S1 | O
   static constexpr int kTmemCols = kOCol + D <= 256 ? 256 : 512;
@@ -122,7 +124,73 @@ struct TcParams {
   int chunk, max_chunks, capacity, max_blocks, num_blocks, max_seqlen;
   float scale_log2;
   int causal;
+  int balanced, n_chunks, B;   // balanced split: n_chunks over the batch (per KV head)
+  int* plan;                   // [B, 3] written by CTA 0 for the combine kernel
 };
+
+// Balanced split: the chunks of this launch and this CTA's (sequence, KV head, chunk),
+// built identically by every CTA from the lengths (integer arithmetic only).  Sequence
+// b gets 1 + floor(L_b (N - B) / sum L) chunks plus one more if its remainder is among
+// the N - B - sum(floor) largest (ties by index), so exactly N chunks in all; its chunk
+// length is ceil(L_b / n_b) rounded up to whole 64-token tiles.  Linear block index
+// i = Hkv * first_b + g * n_b + c is the partial's index.  Lengths outside
+// [1, max_seqlen] count as clamped (such a sequence's rows are reported invalid anyway).
+struct BalancedItem {
+  int b, g, c, chunk;
+};
+__device__ __forceinline__ BalancedItem balanced_item(const TcParams& p, int* plan_smem) {
+  int* len = plan_smem;                                   // [B]
+  int* base = plan_smem + kBalancedMaxB;                  // [B] floor share
+  int* nb = plan_smem + 2 * kBalancedMaxB;                // [B] chunks
+  int* first = plan_smem + 3 * kBalancedMaxB;             // [B] first chunk
+  const int B = p.B, N = p.n_chunks;
+  for (int i = threadIdx.x; i < B; i += blockDim.x) len[i] = min(max(p.seqlens[i], 1), p.max_seqlen);
+  __syncthreads();
+  long long tot = 0;
+  for (int i = 0; i < B; ++i) tot += len[i];
+  const long long spare = N - B;
+  for (int i = threadIdx.x; i < B; i += blockDim.x) base[i] = (int)((long long)len[i] * spare / tot);
+  __syncthreads();
+  long long used = 0;
+  for (int i = 0; i < B; ++i) used += base[i];
+  const long long extra = spare - used;                   // 0 <= extra < B
+  for (int i = threadIdx.x; i < B; i += blockDim.x) {
+    const long long ri = (long long)len[i] * spare % tot;
+    int rank = 0;
+    for (int j = 0; j < B; ++j) {
+      const long long rj = (long long)len[j] * spare % tot;
+      rank += (rj > ri) || (rj == ri && j < i);
+    }
+    nb[i] = 1 + base[i] + (rank < extra ? 1 : 0);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int f = 0;
+    for (int i = 0; i < B; ++i) {
+      first[i] = f;
+      f += nb[i];
+    }
+  }
+  __syncthreads();
+  BalancedItem it;
+  const int id = blockIdx.x;
+  int b = 0;
+  while (b + 1 < B && p.Hkv * first[b + 1] <= id) ++b;
+  const int rem = id - p.Hkv * first[b];
+  it.b = b;
+  it.g = rem / nb[b];
+  it.c = rem - it.g * nb[b];
+  const int per = (len[b] + nb[b] - 1) / nb[b];
+  it.chunk = (per + kTok - 1) / kTok * kTok;
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < B; i += blockDim.x) {
+      const int per_i = (len[i] + nb[i] - 1) / nb[i];
+      p.plan[3 * i] = first[i];
+      p.plan[3 * i + 1] = nb[i];
+      p.plan[3 * i + 2] = (per_i + kTok - 1) / kTok * kTok;
+    }
+  return it;
+}
 
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                         unsigned* status) {
@@ -172,20 +240,36 @@ __global__ void __launch_bounds__(tc_threads<FP8>(), kCtasPerSm)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int c = blockIdx.x % p.max_chunks, rt = blockIdx.x / p.max_chunks, g = blockIdx.y, b = blockIdx.z;
+  int c, rt, g, b, chunk;
+  size_t item;
+  if (p.balanced) {
+    const BalancedItem bi = balanced_item(p, reinterpret_cast<int*>(smem + C::kPlanOff));
+    c = bi.c;
+    rt = 0;
+    g = bi.g;
+    b = bi.b;
+    chunk = bi.chunk;
+    item = blockIdx.x;
+  } else {
+    c = blockIdx.x % p.max_chunks;
+    rt = blockIdx.x / p.max_chunks;
+    g = blockIdx.y;
+    b = blockIdx.z;
+    chunk = p.chunk;
+    item = ((size_t)b * p.Hkv + g) * p.max_chunks + c;
+  }
   const int L = p.seqlens[b];
   // invalid lengths are reported (and their rows made NaN) by the combine kernel
   if (L < p.T || L > p.max_seqlen || (!PAGED && L > p.capacity) ||
       (PAGED && (L + kPageTokens - 1) / kPageTokens > p.max_blocks))
     return;
-  const int tok_begin = c * p.chunk;
+  const int tok_begin = c * chunk;
   if (tok_begin >= L) return;   // the combine reads only chunks that start before L
   const int t0 = rt * p.TT;                      // first token of this row tile
   const int tile_tokens = min(p.TT, p.T - t0);
   const int tile_rows = tile_tokens * p.G;       // live rows: 0 .. tile_rows - 1
-  const size_t item = ((size_t)b * p.Hkv + g) * p.max_chunks + c;
   const size_t row0 = item * p.R + (size_t)t0 * p.G;   // partial row of tile row 0
-  int tok_end = min(tok_begin + p.chunk, L);
+  int tok_end = min(tok_begin + chunk, L);
   if (p.causal) tok_end = min(tok_end, L - p.T + t0 + tile_tokens);   // last token's first invisible key
   if (tok_end <= tok_begin) {
     // no key of this chunk is visible to any row of the tile: an empty partial
@@ -639,11 +723,17 @@ cudaError_t run_tc(const DecodeLaunch& a, const CUtensorMap& tk, const CUtensorM
   p.max_seqlen = a.max_seqlen;
   p.scale_log2 = a.scale * kLog2e;
   p.causal = a.causal;
+  p.balanced = a.balanced;
+  p.n_chunks = a.n_chunks;
+  p.B = a.B;
+  p.plan = a.plan;
+  if (a.balanced && (a.B > kBalancedMaxB || row_tiles != 1 || a.n_chunks < a.B)) return cudaErrorInvalidValue;
   auto kern = decode_tc_kernel<D, PAGED, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   if ((long long)a.max_chunks * row_tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
   dim3 grid(a.max_chunks * row_tiles, a.Hkv, a.B);
+  if (a.balanced) grid = dim3((unsigned)a.n_chunks * a.Hkv);
   kern<<<grid, tc_threads<FP8>(), C::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }

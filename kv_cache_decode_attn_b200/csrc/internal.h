@@ -18,10 +18,30 @@ constexpr int kDecodeTcTile = 64;  // tokens per K/V tile of the tensor-core dec
 // streams at the HBM rate.
 constexpr int kDecodeMmaRows = 16;
 // FP8 caches run the warp-MMA kernels up to this many rows per KV head, and the
-// tensor-core kernel (converting each e4m3 tile to bf16 in shared memory) above.
+// tensor-core kernel (converting each e4m3 tile to f16 in shared memory) above.
 constexpr int kFp8MaxRows = 32;
 // Whether attn_decode runs the tensor-core split kernel for R rows per KV head.
 inline bool decode_uses_tc(int R, bool fp8) { return R > (fp8 ? kFp8MaxRows : kDecodeMmaRows); }
+
+// Balanced split of the tensor-core decode kernel.  With one fixed chunk length the
+// number of chunks of each sequence is its length rounded up, and the total over the
+// batch falls anywhere against the 2 CTAs x SMs slots: measured on B200 (paged Llama
+// decode, 8 x 8 sequence-heads, lengths 32K-131K, 4 seeds), one split count ran at
+// 94-101 % of the HBM copy rate where the items came to just under a whole number of
+// slot waves and at 62-80 % just over one.  The host knows only max_seqlen, so the
+// kernel itself apportions kBalancedItemsPerSlot x slots chunks over the sequences in
+// proportion to their lengths (at least one each, the rest by largest remainder), each
+// sequence cut into its own number of equal chunks.
+constexpr int kDecodeTcCtasPerSm = 2;      // shared memory and TMEM of one tensor-core decode CTA
+constexpr int kBalancedItemsPerSlot = 2;
+constexpr int kBalancedMaxB = 128;         // the plan is built per CTA in shared memory
+// Whether attn_decode with these sizes uses the balanced split (automatic splitting, the
+// tensor-core kernel, one row tile per KV head).
+inline bool decode_balanced(int B, int T, int G, int num_splits, bool fp8) {
+  return num_splits == 0 && B <= kBalancedMaxB && decode_uses_tc(G * T, fp8) && G * T <= 128;
+}
+// Chunks over the whole batch (per KV head) of the balanced split on the current device.
+int decode_balanced_chunks(int B, int Hkv);
 
 // One CTA whose thread waits on an mbarrier nothing arrives at (bounded like every
 // wait of the library) and then sets DEV_TIMEOUT (csrc/selftest.cu).
@@ -42,9 +62,13 @@ struct DecodeLaunch {
   int causal;
   int chunk;          // tokens per split (multiple of kDecodeTile)
   int max_chunks;     // ceil(max_seqlen / chunk)
-  float* part_o;      // [B, Hkv, max_chunks, R, d]
-  float* part_lse;    // [B, Hkv, max_chunks, R]
+  float* part_o;      // [B, Hkv, max_chunks, R, d]; balanced: [n_chunks * Hkv, R, d]
+  float* part_lse;    // [B, Hkv, max_chunks, R];    balanced: [n_chunks * Hkv, R]
   unsigned* status;
+  // balanced split (decode_balanced): chunks over the batch, and the per-sequence plan
+  // (first chunk, chunks, chunk length) the split kernel writes for the combine
+  int balanced = 0, n_chunks = 0;
+  int* plan = nullptr;   // [B, 3]
   int fp8 = 0;                    // k/v hold e4m3 codes with per-KV-head scales
   const float* k_scale = nullptr;  // [Hkv]
   const float* v_scale = nullptr;

@@ -23,6 +23,8 @@ struct SplitParams {
   int chunk, max_chunks, capacity, max_blocks, num_blocks, max_seqlen;
   float scale_log2;
   int causal;
+  int balanced = 0;            // tensor-core balanced split: partials indexed by the plan
+  const int* plan = nullptr;   // [B, 3]: first chunk, chunks, chunk length per sequence
 };
 
 __device__ __forceinline__ bool seqlen_bad(int L, int T, int max_seqlen, bool paged, int capacity, int max_blocks) {

@@ -101,7 +101,9 @@ def test_noalloc_request_that_nearly_fills_its_array():
 def test_noalloc_rejects_requests_beyond_its_array():
     """Needs no GPU: the size check runs before anything touches a device."""
     P = 256
-    B, T, Hq, Hkv, d, msk = 64, 4, 64, 8, 128, 131072
+    # one new token (8 rows per KV head: the warp-MMA kernel's fixed chunking in both the
+    # bf16 and the FP8 layout)
+    B, T, Hq, Hkv, d, msk = 64, 1, 64, 8, 128, 131072
     need = kv.attn_decode_workspace_bytes(B, T, Hq, Hkv, d, msk, 0)
     assert need > kv.ATTN_DECODE_NOALLOC_SCRATCH_BYTES
     st = kv.lib.attn_decode_noalloc(P, P, P, P, None, 0, 0, msk, msk, P, 0, None, B, T, Hq, Hkv, d, 0.1, 1, 0, None)
