@@ -98,6 +98,39 @@ def test_decode_many_rows_per_kv_head(paged, T, Hq, Hkv, d):
     check_lse(lse, lse_ref)
 
 
+@pytest.mark.parametrize("paged", [False, True])
+@pytest.mark.parametrize("B", [100, 129])
+def test_decode_balanced_split_many_sequences(paged, B):
+    """Automatic splitting on the tensor-core kernel apportions the chunks over the
+    sequences by their lengths (B <= 128; B = 129 takes the fixed chunk length): many
+    sequences of very different lengths, some with no cached token at all."""
+    T, Hq, Hkv, d = 8, 16, 2, 128
+    rng = np.random.default_rng(900 + B)
+    lens = [int(x) for x in rng.integers(0, 3000, size=B)]
+    lens[0], lens[1], lens[-1] = 0, 2999, 1
+    case = synth.decode_inputs(B, T, Hq, Hkv, d, 0, 0, seed=901 + B, device="cuda", paged=paged, lengths=lens,
+                               spare_blocks=1)
+    host = host_copy(case)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = run_step(case, T, Hq, Hkv, d, scale)
+    o_ref, lse_ref = oracle_step(host, T, scale)
+    check_o(o, o_ref)
+    check_lse(lse, lse_ref)
+
+
+def test_decode_balanced_split_single_long_sequence():
+    """One sequence: all the batch's chunks go to it (most of the grid's CTAs find their
+    chunk past the end and leave)."""
+    T, Hq, Hkv, d = 4, 32, 4, 128
+    case = synth.decode_inputs(1, T, Hq, Hkv, d, 0, 0, seed=905, device="cuda", paged=True, lengths=[20000])
+    host = host_copy(case)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = run_step(case, T, Hq, Hkv, d, scale)
+    o_ref, lse_ref = oracle_step(host, T, scale)
+    check_o(o, o_ref)
+    check_lse(lse, lse_ref)
+
+
 @pytest.mark.parametrize("num_splits", [1, 2, 3, 7, 40])
 @pytest.mark.parametrize("T", [1, 4])
 def test_decode_split_counts(num_splits, T):
