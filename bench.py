@@ -229,8 +229,14 @@ def append_and_attend(kv, wd, kc, vc, q, k_new, v_new, cache_lens, seqlens, tabl
         ev[3].record(stream)
 
 
+def decode_via_prefill(wd) -> bool:
+    """attn_decode with at least 256 new tokens on a bf16 cache (automatic splitting)
+    runs the prefill kernel's cached form."""
+    return not wd.fp8 and wd.T >= 256
+
+
 def decode_kernel_name(wd, prefill_cache=False) -> str:
-    if prefill_cache:
+    if prefill_cache or decode_via_prefill(wd):
         return "prefill_kernel<128, paged cache>" if wd.paged else "prefill_kernel<128, cache>"
     return f"{decode_kernel(wd)[0]} + decode_combine_kernel"
 
@@ -241,6 +247,8 @@ def decode_kernel(wd):
     8 rows on the transposed-product kernel, up to 32 on the split kernel, more on
     tcgen05 (e4m3 tiles converted to f16 in shared memory)."""
     R = wd.Hq // wd.Hkv * wd.T
+    if decode_via_prefill(wd):
+        return "prefill_kernel<128, paged cache>" if wd.paged else "prefill_kernel<128, cache>", ("prefill.cu",)
     if wd.fp8:
         if R <= 8:
             return "decode_fp8_st_kernel", ("decode_fp8.cu", "split.cuh", "decode.cu")
@@ -421,7 +429,7 @@ def run_ours(args, world, rank, local):
             "e2e": e2e,
             # per step: prefill, append, then decode split + combine (or one attn_prefill_cache launch);
             # the configuration runs are outside the timed region
-            "gpu_launches": (3 if prefill_cache else 4) * K,
+            "gpu_launches": (3 if prefill_cache or decode_via_prefill(wd) else 4) * K,
             "clocks": clocks.summary(),
         }
     if world > 1:

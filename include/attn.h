@@ -169,7 +169,9 @@ ATTN_API size_t attn_decode_workspace_bytes(int B, int T, int Hq, int Hkv, int d
  * the chunk length, and T = seqlens_k[b] is a prefill from scratch.  With
  * R = (Hq / Hkv) * T query rows per KV head, R <= 16 runs on warp-level MMAs;
  * larger R on the tcgen05 tensor cores, in row tiles of whole tokens of at most
- * 128 rows, scores in TMEM.  Hq / Hkv must be <= 128.
+ * 128 rows, scores in TMEM.  With T >= 256 and num_splits == 0 the call runs
+ * attn_prefill_cache's kernel instead (same rows, same length rules; the
+ * workspace is then not written).  Hq / Hkv must be <= 128.
  * Errors: ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED (d, rows per KV head),
  * ATTN_ERR_WORKSPACE, ATTN_ERR_CUDA.  Bad lengths or page ids found on the
  * device set ATTN_DEV_SEQLEN / ATTN_DEV_PAGE_ID and make the affected rows NaN.

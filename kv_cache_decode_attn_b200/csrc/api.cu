@@ -238,6 +238,33 @@ int decode_impl(const void* q, const void* k_cache, const void* v_cache, const f
   if (!workspace || !aligned16(workspace)) return ATTN_ERR_WORKSPACE;
   unsigned* st = status_ptr();
   if (!st) return ATTN_ERR_CUDA;
+  if (!fp8 && num_splits == 0 && T >= kDecodeViaPrefillT && (long long)B * T * Hq <= INT32_MAX) {
+    // a prompt chunk against a cached prefix: the prefill kernel's cached form computes the
+    // same rows (bottom-right causal alignment, the same length rules with max_seqlen_k) faster;
+    // the workspace goes unused
+    PrefillLaunch pa;
+    pa.q = q;
+    pa.k = k_cache;
+    pa.v = v_cache;
+    pa.o = o;
+    pa.o_bf16 = o_dtype == ATTN_BF16;
+    pa.lse = lse;
+    pa.B = B;
+    pa.Hq = Hq;
+    pa.Hkv = Hkv;
+    pa.N = T;
+    pa.d = d;
+    pa.scale = scale;
+    pa.causal = causal;
+    pa.status = st;
+    pa.seqlens = seqlens_k;
+    pa.page_table = page_table;
+    pa.capacity = cache_capacity;
+    pa.max_blocks = max_blocks_per_seq;
+    pa.num_blocks = num_blocks;
+    pa.max_seqlen = max_seqlen_k;
+    return cuda_status(launch_prefill(pa, static_cast<cudaStream_t>(stream)), name);
+  }
   DecodeLaunch a;
   a.q = q;
   a.k = k_cache;

@@ -89,7 +89,15 @@ struct PrefillLaunch {
   const int32_t* seqlens = nullptr;     // [B] keys per sequence, including the N new ones
   const int32_t* page_table = nullptr;  // [B, max_blocks], or nullptr for a contiguous cache
   int capacity = 0, max_blocks = 0, num_blocks = 0;
+  int max_seqlen = 0;   // > 0: lengths above it are invalid too (attn_decode's max_seqlen_k)
 };
+
+// attn_decode with at least this many new tokens (bf16 cache, automatic splitting)
+// runs the prefill kernel's cached form: measured on B200 (Llama heads, 4K-16K cached
+// keys, B 4 and 16, paged and contiguous), the split tensor-core path was faster up to
+// T = 128 (decode 557-867 against 429-618 TFLOP/s) and slower from T = 256 (729-901
+// against 873-1176), where each sequence has whole 256-row query blocks to stream.
+constexpr int kDecodeViaPrefillT = 256;
 
 struct AppendLaunch {
   void* k;

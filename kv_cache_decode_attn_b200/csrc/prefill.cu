@@ -834,6 +834,7 @@ cudaError_t run_prefill(const PrefillLaunch& a, cudaStream_t stream) {
   p.max_blocks = a.max_blocks;
   p.num_blocks = a.num_blocks;
   p.max_keys = KV == KV_PAGED ? a.max_blocks * kPageTokens : (KV == KV_CACHE ? a.capacity : a.N);
+  if (!kDenseKv<KV> && a.max_seqlen > 0 && a.max_seqlen < p.max_keys) p.max_keys = a.max_seqlen;
   cudaError_t qe = queue_slot(&p.next_item, &p.done_ctas);
   if (qe != cudaSuccess) return qe;
   auto kern = prefill_kernel<D, KV>;

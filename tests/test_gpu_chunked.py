@@ -50,6 +50,39 @@ def test_many_new_tokens_parity(paged, T, Hq, Hkv, d, num_splits):
     check_lse(lse, lse_ref)
 
 
+@pytest.mark.parametrize("paged", [False, True])
+def test_many_new_tokens_length_rules(paged):
+    """attn_decode with T >= 256 new tokens (the prefill kernel's cached form) keeps
+    attn_decode's length rules: a length above max_seqlen_k, or below T, gives NaN rows
+    and ATTN_DEV_SEQLEN; the other sequences are exact."""
+    T, Hq, Hkv, d = 256, 4, 2, 64
+    lens = [100, 300, 700]
+    case = synth.decode_inputs(len(lens), T, Hq, Hkv, d, 0, 0, seed=73, device="cuda", paged=paged, lengths=lens,
+                               spare_blocks=2)
+    host = host_copy(case)
+    scale = 1.0 / math.sqrt(d)
+    kc = case.k_pool if paged else case.k_cache
+    vc = case.v_pool if paged else case.v_cache
+    table = None if case.page_table is None else to_dev_i32(case.page_table)
+    kv.kv_append(kc, vc, case.k_new, case.v_new, to_dev_i32(case.cache_lens), page_table=table)
+    o_ref, lse_ref = oracle_step(host, T, scale)
+    o = torch.empty(len(lens), T, Hq, d, device="cuda")
+    lse = torch.empty(len(lens), Hq, T, device="cuda")
+    # every length valid: exact
+    kv.attn_decode(case.q, kc, vc, to_dev_i32(case.seqlens_k), o, lse, page_table=table,
+                   max_seqlen_k=int(case.seqlens_k.max()), scale=scale)
+    check_o(o, o_ref)
+    check_lse(lse, lse_ref)
+    assert kv.attn_get_device_status(clear=True) == 0
+    # sequence 2 above max_seqlen_k (its true length), sequence 0 below T
+    seqlens = [int(x) for x in case.seqlens_k]
+    bad = to_dev_i32([T - 1, seqlens[1], seqlens[2]])
+    kv.attn_decode(case.q, kc, vc, bad, o, lse, page_table=table, max_seqlen_k=seqlens[2] - 1, scale=scale)
+    assert kv.attn_get_device_status(clear=True) & kv.ATTN_DEV_SEQLEN
+    assert torch.isnan(o[0]).all() and torch.isnan(o[2]).all()
+    check_o(o[1:2], o_ref[1:2])
+
+
 @pytest.mark.parametrize("causal", [True, False])
 def test_many_new_tokens_noncausal_and_bf16_out(causal):
     T, Hq, Hkv, d = 200, 16, 2, 128
