@@ -379,20 +379,22 @@ def run_ours(args, world, rank, local):
     pf_kernel_tflops = flops / (pf_ms / K * 1e-3) / 1e12          # per launch, this rank
     dec_kernel_gbs = dbytes / (dec_ms / K * 1e-3) / 1e9
     traffic = load_traffic(args.workload, wd, wp)
-    roof_pf = {"bound": "tensor", "achieved": round(pf_kernel_tflops, 1), "peak": peaks["bf16_tflops"],
-               "unit": "TFLOP/s", "frac": round(pf_kernel_tflops / peaks["bf16_tflops"], 4),
-               "frac_of_sustained": round(pf_kernel_tflops / peaks["bf16_tflops_sustained"], 4),
-               "peak_source": f"{peak_src} (bf16 burst)", "traffic": traffic.get("prefill"),
+    # the kernels of this line are timed inside a long loop of steps: against the sustained
+    # tensor peak (the burst figure is for a kernel timed alone, as in the configuration runs)
+    roof_pf = {"bound": "tensor", "achieved": round(pf_kernel_tflops, 1), "peak": peaks["bf16_tflops_sustained"],
+               "unit": "TFLOP/s", "frac": round(pf_kernel_tflops / peaks["bf16_tflops_sustained"], 4),
+               "frac_of_burst": round(pf_kernel_tflops / peaks["bf16_tflops"], 4),
+               "peak_source": f"{peak_src} (bf16 sustained)", "traffic": traffic.get("prefill"),
                "kernel": f"prefill_kernel<{wp.d}>", "flops_per_launch": flops,
                "launch_ms": round(pf_ms / K, 4)}
     # the decode call is HBM-bound unless its flops per byte pass the ridge (many new tokens: chunked prefill)
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
     dec_kernel_tflops = dflops / (dec_ms / K * 1e-3) / 1e12
     if dflops / dbytes > ridge:
-        roof_dec = {"bound": "tensor", "achieved": round(dec_kernel_tflops, 1), "peak": peaks["bf16_tflops"],
-                    "unit": "TFLOP/s", "frac": round(dec_kernel_tflops / peaks["bf16_tflops"], 4),
-                    "frac_of_sustained": round(dec_kernel_tflops / peaks["bf16_tflops_sustained"], 4),
-                    "peak_source": f"{peak_src} (bf16 burst)", "traffic": traffic.get("decode"),
+        roof_dec = {"bound": "tensor", "achieved": round(dec_kernel_tflops, 1), "peak": peaks["bf16_tflops_sustained"],
+                    "unit": "TFLOP/s", "frac": round(dec_kernel_tflops / peaks["bf16_tflops_sustained"], 4),
+                    "frac_of_burst": round(dec_kernel_tflops / peaks["bf16_tflops"], 4),
+                    "peak_source": f"{peak_src} (bf16 sustained)", "traffic": traffic.get("decode"),
                     "kernel": decode_kernel_name(wd, prefill_cache),
                     "flops_per_launch": dflops, "bytes_per_launch": dbytes, "launch_ms": round(dec_ms / K, 4)}
     else:
