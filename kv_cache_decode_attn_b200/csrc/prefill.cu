@@ -76,7 +76,7 @@ namespace {
 
 constexpr int kBM = 128;          // query rows per tile (two tiles per CTA)
 constexpr int kBN = 128;          // keys per K/V tile
-constexpr int kThreads = 384;     // 8 softmax warps + TMA warp + MMA warp + 2 idle warps (a full warpgroup)
+constexpr int kThreads = 384;     // 8 softmax warps + 2 TMA warps + MMA warp + 1 idle warp (a full warpgroup)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 of the largest allowed p

@@ -88,7 +88,7 @@ def test_fp8_decode_small_parity(paged, T, Hq, Hkv):
 @pytest.mark.parametrize("T,Hq,Hkv", [(5, 8, 1), (8, 64, 8), (16, 64, 8), (33, 8, 2)])
 def test_fp8_decode_many_rows_tensor_core(paged, T, Hq, Hkv):
     """More than 32 query rows per KV head (40, 64, 128, and 132 in two row tiles):
-    the tensor-core kernel, converting each e4m3 tile to bf16 in shared memory."""
+    the tensor-core kernel, converting each e4m3 tile to f16 in shared memory."""
     d = 128
     case = synth.decode_inputs(len(SMALL_LENS), T, Hq, Hkv, d, 0, 0, seed=900 + T * Hq, device="cuda", paged=paged,
                                lengths=SMALL_LENS, spare_blocks=3, fp8=True)
