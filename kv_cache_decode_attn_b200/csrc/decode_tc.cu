@@ -205,11 +205,21 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
 // swizzle the copy applies) into the f16 operand tile (two halves of D/2 columns,
 // kTok rows of 128 bytes, same swizzle), one warp.  Called for d = 128 only: a raw
 // row of D codes is one 128-byte swizzle span.
+// 16-byte shared accesses are served per quarter-warp, one 128-byte wavefront for
+// eight lanes that hit eight different 16-byte bank groups.  So each quarter-warp
+// takes rows 2p and 2p+1 of a row pair, four chunks of each, from opposite halves of
+// d: chunk c of row r sits in bank group c ^ (r & 7) of the raw tile and c' ^ (r & 7)
+// (c' = 2 (c mod 4) or that + 1) of its half of the f16 tile, and the two rows'
+// groups are then disjoint for the load and for both stores.  (Eight chunks of one
+// row put chunks c and c + 4, which land in the two halves at the same offset, on
+// one bank group: every store took two wavefronts.)
 template <int D>
 __device__ __forceinline__ void convert_tile_e4m3(const uint8_t* raw, uint8_t* conv, int lane) {
+  const int hi = (lane >> 2) & 1, v = (lane >> 3) & 1;
 #pragma unroll 4
-  for (int idx = lane; idx < kTok * 8; idx += 32) {
-    const int r = idx >> 3, c = idx & 7;                  // row, 16-code chunk (d = 16c .. 16c+15)
+  for (int k = 0; k < kTok / 4; ++k) {
+    const int r = 2 * (2 * k + (lane >> 4)) + hi;             // row: rows 4k .. 4k+3 per pass
+    const int c = ((hi ^ v) << 2) + (lane & 3);               // 16-code chunk (d = 16c .. 16c+15)
     const uint4 w = *reinterpret_cast<const uint4*>(raw + r * 128 + ((c ^ (r & 7)) << 4));
     uint32_t o[8];
     e4m3x4_to_f16x2x2(w.x, o[0], o[1]);
