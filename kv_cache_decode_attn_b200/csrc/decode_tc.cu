@@ -11,7 +11,8 @@
 // the combine kernel merges.  With the bottom-right mask a row tile only reads
 // keys up to the last one its last token sees.  Warp roles:
 //   warps 0..3  softmax: thread i owns row i (TMEM lane i); warps whose rows are
-//               all >= R stay idle;
+//               all >= R stay idle (FP8 with R <= 64: warps 3 and 2 help convert
+//               the K and V tiles);
 //   warps 4, 6  TMA producers: warp 4 loads Q once and the K tiles, warp 6 the V
 //               tiles, each into its own 2-stage ring with the evict-first L2
 //               policy (64-token tiles; contiguous: one 64-row box per 64
@@ -108,6 +109,8 @@ enum TcBar {
   T_VCFULL,
   T_KCEMPTY,   // FP8: the MMA reading the converted K tile is done
   T_VCEMPTY,
+  T_KHDONE,    // FP8, R <= 64: the helper warp has converted its half of the K tile
+  T_VHDONE,
   T_COUNT
 };
 
@@ -212,12 +215,14 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
 // (c' = 2 (c mod 4) or that + 1) of its half of the f16 tile, and the two rows'
 // groups are then disjoint for the load and for both stores.  (Eight chunks of one
 // row put chunks c and c + 4, which land in the two halves at the same offset, on
-// one bank group: every store took two wavefronts.)
+// one bank group: every store took two wavefronts.)  Pass k converts rows 4k .. 4k+3;
+// the warp runs passes k0 .. k1 - 1 (all kTok / 4 of them, or half when two warps
+// share the tile).
 template <int D>
-__device__ __forceinline__ void convert_tile_e4m3(const uint8_t* raw, uint8_t* conv, int lane) {
+__device__ __forceinline__ void convert_tile_e4m3(const uint8_t* raw, uint8_t* conv, int lane, int k0, int k1) {
   const int hi = (lane >> 2) & 1, v = (lane >> 3) & 1;
 #pragma unroll 4
-  for (int k = 0; k < kTok / 4; ++k) {
+  for (int k = k0; k < k1; ++k) {
     const int r = 2 * (2 * k + (lane >> 4)) + hi;             // row: rows 4k .. 4k+3 per pass
     const int c = ((hi ^ v) << 2) + (lane & 3);               // 16-code chunk (d = 16c .. 16c+15)
     const uint4 w = *reinterpret_cast<const uint4*>(raw + r * 128 + ((c ^ (r & 7)) << 4));
@@ -289,6 +294,9 @@ __global__ void __launch_bounds__(tc_threads<FP8>(), kCtasPerSm)
   }
   const int n_tiles = (tok_end - tok_begin + kTok - 1) / kTok;
   const int active_warps = (tile_rows + 31) / 32;
+  // FP8 with at most 64 rows: softmax warps 2 and 3 are free and convert the second half
+  // of every K (warp 3) and V (warp 2) tile beside the producers
+  const bool conv_split = FP8 && active_warps <= 2;
   float scale_log2 = p.scale_log2, v_mul = 1.f;   // FP8: K scale in the exponent, V scale on O
   if constexpr (FP8) {
     const float ks = __ldg(p.k_scale + g), vs = __ldg(p.v_scale + g);
@@ -323,6 +331,10 @@ __global__ void __launch_bounds__(tc_threads<FP8>(), kCtasPerSm)
     mbar_init(&bars[T_VCFULL], 1);
     mbar_init(&bars[T_KCEMPTY], 1);
     mbar_init(&bars[T_VCEMPTY], 1);
+    if (FP8) {
+      mbar_init(&bars[T_KHDONE], 1);
+      mbar_init(&bars[T_VHDONE], 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -352,7 +364,9 @@ __global__ void __launch_bounds__(tc_threads<FP8>(), kCtasPerSm)
     // Lane 0 copies raw e4m3 tiles into a 2-stage ring; the whole warp converts each
     // raw tile into the one f16 operand tile once the MMA has finished reading the
     // previous one, then refills the raw stage it has just read.  Warp 7 handles K
-    // (and Q), warp 6 V; warp 4 has no work.
+    // (and Q), warp 6 V; warp 4 has no work.  With conv_split the warp converts rows
+    // 0 .. kTok/2 - 1 and its helper (below) the rest; the tile is published, and its raw
+    // stage refilled, once the helper has arrived on its barrier for that tile.
     const bool is_k = warp == 7;
     const CUtensorMap* map = is_k ? &tmK : &tmV;
     uint8_t* raw_ring = smem + (is_k ? C::kRawKOff : C::kRawVOff);
@@ -418,9 +432,12 @@ __global__ void __launch_bounds__(tc_threads<FP8>(), kCtasPerSm)
     for (int i = 0; ok && i < n_tiles; ++i) {
       if (!tc_wait(&bars[full0 + i % kStages], (i / kStages) & 1, abort_flag, p.status)) break;
       if (i > 0 && !tc_wait(cempty, (i - 1) & 1, abort_flag, p.status)) break;
-      convert_tile_e4m3<D>(raw_ring + (i % kStages) * C::kRawBytes, conv, lane);
+      convert_tile_e4m3<D>(raw_ring + (i % kStages) * C::kRawBytes, conv, lane, 0, conv_split ? kTok / 8 : kTok / 4);
       fence_proxy_async_smem();       // the converted tile is read by the MMAs (async proxy)
       __syncwarp();
+      // the helper finishes tile i before the MMA of tile i can release the converted
+      // tile, so its barrier is never more than one phase ahead of this wait
+      if (conv_split && !tc_wait(&bars[is_k ? T_KHDONE : T_VHDONE], i & 1, abort_flag, p.status)) break;
       if (lane == 0) {
         mbar_arrive(cfull);
         if (i + kStages < n_tiles) {   // the raw stage just read takes the tile kStages ahead
@@ -434,6 +451,25 @@ __global__ void __launch_bounds__(tc_threads<FP8>(), kCtasPerSm)
     if (lane == 0) {
       if (is_k) mbar_wait(&bars[T_Q], 0);
       for (int i = max(0, issued - kStages); i < issued; ++i) mbar_wait(&bars[full0 + i % kStages], (i / kStages) & 1);
+    }
+  } else if (conv_split && (warp == 3 || warp == 2)) {
+    // ------------------------------------------------ FP8 conversion helpers (R <= 64)
+    // Rows kTok/2 .. kTok - 1 of every raw tile: the same waits as the producer's
+    // conversion (raw tile landed, previous converted tile released by the MMA), then
+    // one arrival per tile.  The producer refills the raw stage only after that arrival.
+    const bool is_k = warp == 3;
+    const uint8_t* raw_ring = smem + (is_k ? C::kRawKOff : C::kRawVOff);
+    uint8_t* conv = smem + (is_k ? C::kKOff : C::kVOff);
+    const int full0 = is_k ? T_KFULL : T_VFULL;
+    uint64_t* cempty = &bars[is_k ? T_KCEMPTY : T_VCEMPTY];
+    uint64_t* hdone = &bars[is_k ? T_KHDONE : T_VHDONE];
+    for (int i = 0; i < n_tiles; ++i) {
+      if (!tc_wait(&bars[full0 + i % kStages], (i / kStages) & 1, abort_flag, p.status)) break;
+      if (i > 0 && !tc_wait(cempty, (i - 1) & 1, abort_flag, p.status)) break;
+      convert_tile_e4m3<D>(raw_ring + (i % kStages) * C::kRawBytes, conv, lane, kTok / 8, kTok / 4);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(hdone);
     }
   } else if (!FP8 && (warp == 4 || warp == 6)) {
     // ------------------------------------------------------------- TMA producers
