@@ -213,7 +213,8 @@ def test_fp8_decode_ignores_nan_codes_past_the_end(T, Hq, Hkv):
         check_lse(lse, lse_ref)
 
 
-@pytest.mark.parametrize("T,Hq,Hkv", [(4, 32, 4), (2, 16, 4)])
+# (8, 64, 8): 64 rows per KV head, the tensor-core form with the conversion helper warps
+@pytest.mark.parametrize("T,Hq,Hkv", [(4, 32, 4), (2, 16, 4), (8, 64, 8)])
 def test_fp8_paged_equals_contiguous_bitwise(T, Hq, Hkv):
     d = 128
     lens = [1, 77, 1000, 4000]
