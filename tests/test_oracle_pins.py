@@ -62,6 +62,18 @@ def test_kv_bytes_units_printed_on_pages():
     assert oracle.kv_cache_bytes(80, 1, 32768, 64, 128, 2) == 8 * oracle.kv_cache_bytes(80, 1, 32768, 8, 128, 2)
 
 
+def test_concurrent_request_figures_printed_on_the_page():
+    # [BEE-30062], GQA section, prints 2,500 (8 KV heads) and 625 (32 KV heads) requests of 4K
+    # context in 40 GB.  Those are 40,000 MB over one request's per-layer K+V size taken in MB
+    # (16 and 64: the page's own "16 MB" is 16 MiB), i.e. the printed figures leave the layer
+    # factor out; the oracle's byte count reproduces them exactly under that reading.
+    for n_kv_heads, printed in ((8, 2500), (32, 625)):
+        per_layer = oracle.kv_cache_bytes(1, 1, 4096, n_kv_heads, 128, 2)
+        assert per_layer % 2**20 == 0
+        assert 40_000 // (per_layer // 2**20) == printed
+        assert 40_000 % (per_layer // 2**20) == 0
+
+
 def test_kv_bytes_errors():
     assert oracle.kv_cache_bytes(0, 1, 1, 1, 1, 1) == -1
     assert oracle.kv_cache_bytes(1, 1, -5, 1, 1, 1) == -1
