@@ -58,6 +58,24 @@ def test_workspace_bytes():
     assert kv.attn_decode_workspace_bytes(2, 1, 8, 2, 64, 5000, 10) >= kv.attn_decode_workspace_bytes(2, 1, 8, 2, 64, 5000, 2)
 
 
+def test_workspace_bytes_balanced_split():
+    # Automatic splitting on the tensor-core path with at most 128 sequences apportions a fixed
+    # number of chunks, two per CTA slot (2 CTAs on each of a B200's 148 SMs, assumed on a host
+    # without a device) per KV head, whatever the cache length: the workspace holds every chunk's
+    # partial O and LSE rows plus the B x 3 plan, and does not grow with max_seqlen_k.
+    B, T, Hq, Hkv, d = 8, 8, 64, 8, 128
+    sizes = {kv.attn_decode_workspace_bytes(B, T, Hq, Hkv, d, L) for L in (4096, 32768, 131072, 1 << 20)}
+    assert len(sizes) == 1
+    n = sizes.pop()
+    chunks = 2 * 2 * 148 // Hkv
+    need = chunks * Hkv * (Hq // Hkv) * T * (d + 1) * 4 + B * 3 * 4
+    assert need <= n <= need + 1024
+    # past 128 sequences the launch takes one chunk length, and the workspace follows the length
+    assert kv.attn_decode_workspace_bytes(129, T, Hq, Hkv, d, 131072) > kv.attn_decode_workspace_bytes(129, T, Hq, Hkv, d, 4096)
+    # one row per KV head (T = 1, the warp-level kernel): chunking follows the length as well
+    assert kv.attn_decode_workspace_bytes(B, 1, Hq, Hkv, d, 1 << 20) > kv.attn_decode_workspace_bytes(B, 1, Hq, Hkv, d, 4096)
+
+
 # Host-side argument checks return before anything touches a device, so they
 # can run here with dummy (never dereferenced) pointers.
 P = 256   # a fake, 16-byte aligned non-null pointer value
