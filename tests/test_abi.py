@@ -72,7 +72,7 @@ def test_workspace_bytes_balanced_split():
     assert need <= n <= need + 1024
     # past 128 sequences the launch takes one chunk length, and the workspace follows the length
     assert kv.attn_decode_workspace_bytes(129, T, Hq, Hkv, d, 131072) > kv.attn_decode_workspace_bytes(129, T, Hq, Hkv, d, 4096)
-    # one row per KV head (T = 1, the warp-level kernel): chunking follows the length as well
+    # T = 1 (8 rows per KV head, the warp-level kernels): chunking follows the length as well
     assert kv.attn_decode_workspace_bytes(B, 1, Hq, Hkv, d, 1 << 20) > kv.attn_decode_workspace_bytes(B, 1, Hq, Hkv, d, 4096)
 
 
