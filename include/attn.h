@@ -129,7 +129,8 @@ ATTN_API int attn_prefill_cache(const void* q, const void* k_cache, const void* 
  * attn_decode_workspace_bytes -- bytes of device workspace attn_decode and
  * attn_decode_fp8 need for these sizes (the per-chunk partial outputs and
  * log-sum-exps of the split along the keys; the larger of the two, whose key
- * chunking differs).  num_splits as for attn_decode.  Returns 0 for invalid sizes.
+ * chunking differs).  num_splits as for attn_decode.  Returns 0 for invalid sizes,
+ * including max_seqlen_k above 2^30.
  */
 ATTN_API size_t attn_decode_workspace_bytes(int B, int T, int Hq, int Hkv, int d, int max_seqlen_k, int num_splits);
 
@@ -154,7 +155,8 @@ ATTN_API size_t attn_decode_workspace_bytes(int B, int T, int Hq, int Hkv, int d
  *   max_blocks_per_seq, num_blocks   paged sizes (ignored when contiguous)
  *   cache_capacity  contiguous token capacity per sequence (ignored when paged)
  *   max_seqlen_k    host-side upper bound on every seqlens_k[b] (sizes the split
- *                   grid and the workspace); 0 = the cache capacity
+ *                   grid and the workspace), at most 2^30 (ATTN_ERR_UNSUPPORTED
+ *                   above); 0 = the cache capacity, capped at 2^30
  *   o           device [B, T, Hq, d] of o_dtype;  lse  device fp32 [B, Hq, T] or NULL
  *   scale, causal   as for attn_prefill; causal with T == 1 equals non-causal
  *   num_splits  0 = automatic chunking (on the tensor-core kernel with one row

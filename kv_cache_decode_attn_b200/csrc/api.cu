@@ -88,11 +88,12 @@ struct DecodeLayout {
 bool decode_layout(int B, int T, int Hq, int Hkv, int d, int max_seqlen_k, int num_splits, bool fp8,
                    DecodeLayout* out) {
   if (B < 1 || T < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || max_seqlen_k < 1 || num_splits < 0) return false;
+  if (max_seqlen_k > kMaxDecodeSeqlen) return false;
   if (d != 64 && d != 128) return false;
   DecodeLayout L;
   L.R = (Hq / Hkv) * T;
   L.chunk = decode_chunk_tokens(B, T, Hq / Hkv, Hkv, max_seqlen_k, num_splits, fp8);
-  L.max_chunks = (max_seqlen_k + L.chunk - 1) / L.chunk;
+  L.max_chunks = (int)(((long long)max_seqlen_k + L.chunk - 1) / L.chunk);
   L.balanced = decode_balanced(B, T, Hq / Hkv, num_splits, fp8) ? 1 : 0;
   L.n_chunks = 0;
   size_t items = (size_t)B * Hkv * L.max_chunks;
@@ -221,8 +222,9 @@ int decode_impl(const void* q, const void* k_cache, const void* v_cache, const f
     if ((long long)B * cache_capacity > INT32_MAX) return ATTN_ERR_UNSUPPORTED;
     capacity_tokens = cache_capacity;
   }
-  if (max_seqlen_k == 0) max_seqlen_k = capacity_tokens;
+  if (max_seqlen_k == 0) max_seqlen_k = std::min(capacity_tokens, kMaxDecodeSeqlen);
   if (max_seqlen_k < T || max_seqlen_k > capacity_tokens) return ATTN_ERR_INVALID_ARG;
+  if (max_seqlen_k > kMaxDecodeSeqlen) return ATTN_ERR_UNSUPPORTED;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (Hq / Hkv > 128) return ATTN_ERR_UNSUPPORTED;                       // one token's heads must fit a row tile
   if (fp8 && d != 128) return ATTN_ERR_UNSUPPORTED;

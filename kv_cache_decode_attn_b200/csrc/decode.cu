@@ -624,7 +624,7 @@ cudaError_t run_split(const CUtensorMap& tk, const CUtensorMap& tv, const SplitP
 int decode_chunk_tokens(int B, int T, int G, int Hkv, int max_seqlen, int num_splits, bool fp8) {
   int chunk;
   if (num_splits > 0) {
-    chunk = (max_seqlen + num_splits - 1) / num_splits;
+    chunk = (int)(((long long)max_seqlen + num_splits - 1) / num_splits);
   } else {
     // Long chunks stream longer and leave fewer partials to merge; short ones
     // balance the grid.  Measured on B200: the warp-MMA kernel (2 CTAs per SM)
@@ -641,7 +641,7 @@ int decode_chunk_tokens(int B, int T, int G, int Hkv, int max_seqlen, int num_sp
     const bool full_tiles = decode_tc_tile_tokens(T, G) * G > 64;
     const long long target = tc ? (full_tiles ? 640 : 1280) : (fp8 && R <= 8 ? 3072 : 2048);
     chunk = tc ? 16384 : 4096;
-    while (chunk > 256 && units * ((max_seqlen + chunk - 1) / chunk) < target) chunk >>= 1;
+    while (chunk > 256 && units * (((long long)max_seqlen + chunk - 1) / chunk) < target) chunk >>= 1;
   }
   // a multiple of both kernels' tiles
   chunk = ((chunk + kDecodeTcTile - 1) / kDecodeTcTile) * kDecodeTcTile;

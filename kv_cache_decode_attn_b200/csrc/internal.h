@@ -34,6 +34,9 @@ inline bool decode_uses_tc(int R, bool fp8) { return R > (fp8 ? kFp8MaxRows : kD
 // sequence cut into its own number of equal chunks.
 constexpr int kDecodeTcCtasPerSm = 2;      // shared memory and TMEM of one tensor-core decode CTA
 constexpr int kBalancedItemsPerSlot = 2;
+// Longest key range one decode call accepts (max_seqlen_k): keeps every token offset,
+// chunk start and chunk end of the decode kernels inside int.
+constexpr int kMaxDecodeSeqlen = 1 << 30;
 constexpr int kBalancedMaxB = 128;         // the plan is built per CTA in shared memory
 // Whether attn_decode with these sizes uses the balanced split (automatic splitting, the
 // tensor-core kernel, one row tile per KV head).

@@ -76,6 +76,21 @@ def test_workspace_bytes_balanced_split():
     assert kv.attn_decode_workspace_bytes(B, 1, Hq, Hkv, d, 1 << 20) > kv.attn_decode_workspace_bytes(B, 1, Hq, Hkv, d, 4096)
 
 
+def test_workspace_bytes_length_limit():
+    # max_seqlen_k is bounded by 2^30 (every token offset and chunk end of the kernels stays in
+    # int); up to it the size is that of the chunks the length needs, above it 0 (unsupported)
+    for args in ((1, 1, 8, 1, 64), (8, 8, 64, 8, 128), (2, 4, 32, 8, 128)):
+        n = kv.attn_decode_workspace_bytes(*args, 1 << 30)
+        assert 0 < n < 1 << 40
+        for L in ((1 << 30) + 1, 2**31 - 1):
+            assert kv.attn_decode_workspace_bytes(*args, L) == 0
+            assert kv.attn_decode_workspace_bytes(*args, L, 3) == 0
+    # 3 splits of 2^30 keys: three chunks of the 8 rows' partials (fp32 O of d = 64, then the LSE
+    # rows, the end rounded up to 256 bytes)
+    o_bytes, lse_bytes = 3 * 8 * 64 * 4, 3 * 8 * 4
+    assert kv.attn_decode_workspace_bytes(1, 1, 8, 1, 64, 1 << 30, 3) == (o_bytes + lse_bytes + 255) // 256 * 256
+
+
 # Host-side argument checks return before anything touches a device, so they
 # can run here with dummy (never dereferenced) pointers.
 P = 256   # a fake, 16-byte aligned non-null pointer value
@@ -117,6 +132,8 @@ def test_decode_rejects_bad_arguments():
     assert call(wsb=16) == kv.ATTN_ERR_WORKSPACE
     assert call(ns=-1) == kv.ATTN_ERR_INVALID_ARG
     assert call(causal=2) == kv.ATTN_ERR_INVALID_ARG
+    # a paged capacity above 2^30 tokens: a bound beyond 2^30 is unsupported
+    assert call(pt=P, mb=(1 << 26) + 1, nb=1, msk=(1 << 30) + 1) == kv.ATTN_ERR_UNSUPPORTED
 
 
 def test_append_rejects_bad_arguments():
@@ -146,6 +163,7 @@ def test_decode_fp8_rejects_bad_arguments():
     assert call(Hq=256, Hkv=1) == kv.ATTN_ERR_UNSUPPORTED      # one token's heads exceed a 128-row tile
     assert call(wsb=16) == kv.ATTN_ERR_WORKSPACE
     assert call(T=4, msk=3) == kv.ATTN_ERR_INVALID_ARG
+    assert call(pt=P, mb=(1 << 26) + 1, nb=1, msk=(1 << 30) + 1) == kv.ATTN_ERR_UNSUPPORTED
 
 
 def test_append_fp8_rejects_bad_arguments():
